@@ -1,0 +1,400 @@
+"""Pins that tie the fp64 oracle to something other than itself.
+
+Each pin is a plain function taking a loaded oracle library (ctypes handle) and
+raising AssertionError on a mismatch.  ``test_oracle_pins.py`` runs them on the
+real oracle; ``test_oracle_mutants.py`` runs them on copies of the oracle with a
+planted mistake and requires that at least one pin fails for every mistake.
+
+What pins what:
+  * worked example  -- the numbers printed on the "FlashAttention" explainer
+    page (ozercemkelahmet.com), "A worked example" / "Online softmax by hand"
+    (tests/golden/worked_example.json): exponent values, normaliser, and the
+    block-merge rule, all in the page's notation.
+  * uniform scores  -- Q = 0 makes every visible weight equal, so O is the mean
+    of V over the visible key range and LSE = ln(count): a closed form that pins
+    the mask (inclusive window bounds, causal override, sequence boundaries).
+  * two keys        -- softmax of two scores is the logistic function
+    (scipy.special.expit) and the LSE is numpy.logaddexp.
+  * hard limit      -- a very large scale turns softmax into argmax.
+  * single key / causal row 0 -- O = v_0, LSE = scale * q.k_0.
+  * invariants      -- constant V, rows summing to one, key permutation
+    (non-causal), window >= N-1 equals causal, packed == separate calls,
+    grouped-query == key/value heads repeated per query head.
+  * library routine -- torch.nn.functional.scaled_dot_product_attention in
+    float64 on the CPU with a band mask built by torch.triu / torch.tril (the
+    page's own causal-mask recipe in "Checking correctness"), and
+    torch.logsumexp for the LSE.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bf16(x) -> torch.Tensor:
+    t = torch.as_tensor(np.asarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16)
+
+
+def _run(lib, q, k, v, **kw):
+    """q [B,N,Hq,d] / k,v [B,N,Hkv,d] (or packed [T,H,d]) bf16 tensors."""
+    return oracle.attn_fwd(W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v), lib=lib, **kw)
+
+
+def _f64(t: torch.Tensor) -> np.ndarray:
+    return t.to(torch.float64).numpy()
+
+
+# --------------------------------------------------------------------------
+# worked example from the page
+# --------------------------------------------------------------------------
+def pin_worked_example(lib):
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    s = g["scores"]
+    n = len(s)
+    half_ulp = 0.5 * 10.0 ** (-g["printed_decimals"])
+    d = 4
+    # q = e_0, k_j = s_j e_0 so that q.k_j = s_j; v_j = e_j so that O = the weights.
+    q = np.zeros((1, n, 1, d), np.float32)
+    q[0, :, 0, 0] = 1.0
+    k = np.zeros((1, n, 1, d), np.float32)
+    k[0, :, 0, 0] = s
+    v = np.zeros((1, n, 1, d), np.float32)
+    for j in range(n):
+        v[0, j, 0, j] = 1.0
+    o, lse, nvis = _run(lib, _bf16(q), _bf16(k), _bf16(v), B=1, Hq=1, Hkv=1, N=n, d=d,
+                        scale=1.0, causal=False)
+    M = g["direct"]["max"]
+    Z = math.exp(lse[0, 0, 0] - M)
+    # direct computation: the normaliser and each exponent relative to the max
+    assert abs(Z - g["direct"]["sum"]) <= half_ulp, (Z, g["direct"]["sum"])
+    for j in range(n):
+        assert abs(o[0, 0, j] * Z - g["direct"]["exps"][j]) <= half_ulp, (j, o[0, 0, j] * Z)
+    # online: the page's final sum adds two rounded terms
+    assert abs(Z - g["online_final_sum"]) <= 2 * half_ulp
+    assert nvis[0, 0, 0] == n
+    # block by block: run the oracle on each key block alone
+    lse_blocks = []
+    for blk, ref in zip(g["blocks"], (g["block1"], g["block2"])):
+        nb = len(blk)
+        kb = np.ascontiguousarray(k[:, blk])
+        vb = np.zeros((1, nb, 1, d), np.float32)
+        for jj in range(nb):
+            vb[0, jj, 0, jj] = 1.0
+        qb = np.ascontiguousarray(q[:, :nb])
+        ob, lb, _ = _run(lib, _bf16(qb), _bf16(kb), _bf16(vb), B=1, Hq=1, Hkv=1, N=nb, d=d,
+                         scale=1.0, causal=False)
+        Zb = math.exp(lb[0, 0, 0] - ref["max"])
+        assert abs(Zb - ref["sum"]) <= half_ulp, (Zb, ref["sum"])
+        for jj in range(nb):
+            assert abs(ob[0, 0, jj] * Zb - ref["exps"][jj]) <= half_ulp
+        lse_blocks.append(lb[0, 0, 0])
+    # the rescale step: block 1's sum times exp(m1 - m2) is the page's 0.154
+    rescale = math.exp(g["block1"]["max"] - g["block2"]["max"])
+    assert abs(rescale - g["rescale_factor"]) <= half_ulp
+    assert abs(math.exp(lse_blocks[0] - M) - g["rescaled_block1_sum"]) <= half_ulp
+    # merging the two partial results by the same rule gives the whole row
+    merged = np.logaddexp(lse_blocks[0], lse_blocks[1])
+    assert abs(merged - lse[0, 0, 0]) <= 1e-12
+
+
+# --------------------------------------------------------------------------
+# closed forms
+# --------------------------------------------------------------------------
+def _visible_range(i, L, left, right, causal):
+    """Closed form of the visible key range of row i (inclusive ends)."""
+    if causal:
+        right = 0
+    lo = 0 if left < 0 else max(0, i - left)
+    hi = L - 1 if right < 0 else min(L - 1, i + right)
+    return lo, hi
+
+
+MASK_CASES = [
+    # (N, causal, left, right)
+    (13, False, -1, -1),
+    (13, True, -1, -1),
+    (13, True, 3, 0),
+    (13, False, 2, 5),
+    (13, False, 0, 0),
+    (13, False, -1, 2),
+    (13, False, 4, -1),
+    (13, True, 4, 7),  # causal wins over a positive right window
+    (1, True, -1, -1),
+]
+
+
+def pin_uniform_scores(lib):
+    rng = np.random.default_rng(11)
+    d = 8
+    for (N, causal, left, right) in MASK_CASES:
+        q = np.zeros((1, N, 2, d), np.float32)
+        k = rng.standard_normal((1, N, 1, d)).astype(np.float32)
+        v = rng.integers(-8, 9, size=(1, N, 1, d)).astype(np.float32)  # exact in bf16
+        o, lse, nvis = _run(lib, _bf16(q), _bf16(k), _bf16(v), B=1, Hq=2, Hkv=1, N=N, d=d,
+                            scale=0.7, causal=causal, window_left=left, window_right=right)
+        for h in range(2):
+            for i in range(N):
+                lo, hi = _visible_range(i, N, left, right, causal)
+                cnt = hi - lo + 1
+                assert nvis[0, h, i] == cnt, ((N, causal, left, right), i, nvis[0, h, i], cnt)
+                mean = v[0, lo:hi + 1, 0, :].astype(np.float64).mean(axis=0)
+                assert np.allclose(o[i, h], mean, rtol=0, atol=1e-13), ((N, causal, left, right), i)
+                assert abs(lse[0, h, i] - math.log(cnt)) <= 1e-13
+
+
+def pin_uniform_scores_packed(lib):
+    rng = np.random.default_rng(12)
+    d = 4
+    lens = [5, 1, 9, 3]
+    cu = W.cumulative(lens)
+    T = cu[-1]
+    for (causal, left, right) in [(True, -1, -1), (False, -1, -1), (True, 2, 0), (False, 1, 3)]:
+        q = np.zeros((T, 3, d), np.float32)
+        k = rng.standard_normal((T, 3, d)).astype(np.float32)
+        v = rng.integers(-8, 9, size=(T, 3, d)).astype(np.float32)
+        o, lse, nvis = _run(lib, _bf16(q), _bf16(k), _bf16(v), B=len(lens), Hq=3, Hkv=3, N=T,
+                            d=d, scale=1.0, causal=causal, window_left=left,
+                            window_right=right, cu_seqlens=cu)
+        for b, L in enumerate(lens):
+            for h in range(3):
+                for i in range(L):
+                    lo, hi = _visible_range(i, L, left, right, causal)
+                    t0 = cu[b]
+                    mean = v[t0 + lo:t0 + hi + 1, h, :].astype(np.float64).mean(axis=0)
+                    assert np.allclose(o[t0 + i, h], mean, rtol=0, atol=1e-13), (b, h, i)
+                    assert nvis[h, t0 + i] == hi - lo + 1
+                    assert abs(lse[h, t0 + i] - math.log(hi - lo + 1)) <= 1e-13
+
+
+def pin_two_keys(lib):
+    from scipy.special import expit
+    rng = np.random.default_rng(13)
+    d = 16
+    q = _bf16(rng.standard_normal((1, 2, 1, d)))
+    k = _bf16(rng.standard_normal((1, 2, 1, d)))
+    v = _bf16(rng.standard_normal((1, 2, 1, d)))
+    scale = 0.25
+    o, lse, _ = _run(lib, q, k, v, B=1, Hq=1, Hkv=1, N=2, d=d, scale=scale, causal=False)
+    qf, kf, vf = _f64(q)[0, :, 0], _f64(k)[0, :, 0], _f64(v)[0, :, 0]
+    for i in range(2):
+        s0 = scale * float(np.dot(qf[i], kf[0]))
+        s1 = scale * float(np.dot(qf[i], kf[1]))
+        w1 = float(expit(s1 - s0))
+        expect = (1.0 - w1) * vf[0] + w1 * vf[1]
+        assert np.allclose(o[i, 0], expect, rtol=0, atol=1e-12), i
+        assert abs(lse[0, 0, i] - np.logaddexp(s0, s1)) <= 1e-12
+
+
+def pin_hard_limit(lib):
+    # distinct integer scores times a huge scale: softmax -> one-hot at argmax
+    N, d = 6, 8
+    rng = np.random.default_rng(14)
+    q = np.zeros((1, N, 1, d), np.float32)
+    q[..., 0] = 1.0
+    perm = rng.permutation(N).astype(np.float32)
+    k = np.zeros((1, N, 1, d), np.float32)
+    k[0, :, 0, 0] = perm
+    v = rng.integers(-5, 6, size=(1, N, 1, d)).astype(np.float32)
+    o, lse, _ = _run(lib, _bf16(q), _bf16(k), _bf16(v), B=1, Hq=1, Hkv=1, N=N, d=d,
+                     scale=80.0, causal=False)
+    j = int(np.argmax(perm))
+    for i in range(N):
+        assert np.allclose(o[i, 0], v[0, j, 0], rtol=0, atol=1e-12)
+        assert abs(lse[0, 0, i] - 80.0 * perm[j]) <= 1e-9
+
+
+def pin_single_key_and_row0(lib):
+    rng = np.random.default_rng(15)
+    d = 32
+    q = _bf16(rng.standard_normal((2, 5, 2, d)))
+    k = _bf16(rng.standard_normal((2, 5, 2, d)))
+    v = _bf16(rng.standard_normal((2, 5, 2, d)))
+    scale = 0.3
+    # causal: row 0 sees only key 0
+    o, lse, _ = _run(lib, q, k, v, B=2, Hq=2, Hkv=2, N=5, d=d, scale=scale, causal=True)
+    o = o.reshape(2, 5, 2, d)
+    qf, kf, vf = _f64(q), _f64(k), _f64(v)
+    for b in range(2):
+        for h in range(2):
+            assert np.array_equal(o[b, 0, h], vf[b, 0, h])
+            assert abs(lse[b, h, 0] - scale * float(np.dot(qf[b, 0, h], kf[b, 0, h]))) <= 1e-12
+    # N = 1
+    o1, lse1, _ = _run(lib, q[:, :1].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous(),
+                       B=2, Hq=2, Hkv=2, N=1, d=d, scale=scale, causal=False)
+    o1 = o1.reshape(2, 1, 2, d)
+    assert np.array_equal(o1[:, 0], vf[:, 0])
+
+
+# --------------------------------------------------------------------------
+# invariants
+# --------------------------------------------------------------------------
+def pin_constant_v_and_row_sums(lib):
+    rng = np.random.default_rng(16)
+    N, d = 40, 16
+    q = _bf16(rng.standard_normal((1, N, 2, d)) * 2)
+    k = _bf16(rng.standard_normal((1, N, 2, d)) * 2)
+    c = rng.integers(-4, 5, size=(d,)).astype(np.float32)
+    v = _bf16(np.broadcast_to(c, (1, N, 2, d)).copy())
+    ones = _bf16(np.ones((1, N, 2, d), np.float32))
+    for causal, left, right in [(False, -1, -1), (True, -1, -1), (False, 5, 3)]:
+        o, _, _ = _run(lib, q, k, v, B=1, Hq=2, Hkv=2, N=N, d=d, scale=0.5, causal=causal,
+                       window_left=left, window_right=right)
+        assert np.allclose(o, np.broadcast_to(c, o.shape), rtol=0, atol=1e-12)
+        o1, _, _ = _run(lib, q, k, ones, B=1, Hq=2, Hkv=2, N=N, d=d, scale=0.5, causal=causal,
+                        window_left=left, window_right=right)
+        assert np.abs(o1 - 1.0).max() <= 1e-12  # rows of P sum to one
+
+
+def pin_key_permutation(lib):
+    rng = np.random.default_rng(17)
+    N, d = 33, 16
+    q = _bf16(rng.standard_normal((1, N, 1, d)))
+    k = _bf16(rng.standard_normal((1, N, 1, d)))
+    v = _bf16(rng.standard_normal((1, N, 1, d)))
+    perm = torch.as_tensor(rng.permutation(N))
+    o, lse, _ = _run(lib, q, k, v, B=1, Hq=1, Hkv=1, N=N, d=d, scale=0.4, causal=False)
+    op, lsep, _ = _run(lib, q, k[:, perm].contiguous(), v[:, perm].contiguous(), B=1, Hq=1,
+                       Hkv=1, N=N, d=d, scale=0.4, causal=False)
+    assert np.abs(o - op).max() <= 1e-12
+    assert np.abs(lse - lsep).max() <= 1e-12
+
+
+def pin_window_equals_causal(lib):
+    rng = np.random.default_rng(18)
+    N, d = 37, 8
+    q = _bf16(rng.standard_normal((2, N, 2, d)))
+    k = _bf16(rng.standard_normal((2, N, 1, d)))
+    v = _bf16(rng.standard_normal((2, N, 1, d)))
+    base, lb, _ = _run(lib, q, k, v, B=2, Hq=2, Hkv=1, N=N, d=d, scale=0.5, causal=True)
+    for left in (N - 1, N, 5 * N):
+        o, l, _ = _run(lib, q, k, v, B=2, Hq=2, Hkv=1, N=N, d=d, scale=0.5, causal=False,
+                       window_left=left, window_right=0)
+        assert np.array_equal(o, base) and np.array_equal(l, lb)
+
+
+def pin_packed_equals_separate(lib):
+    rng = np.random.default_rng(19)
+    lens = [7, 1, 12, 4]
+    cu = W.cumulative(lens)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 8
+    q = _bf16(rng.standard_normal((T, Hq, d)))
+    k = _bf16(rng.standard_normal((T, Hkv, d)))
+    v = _bf16(rng.standard_normal((T, Hkv, d)))
+    for causal, left, right in [(True, -1, -1), (False, -1, -1), (False, 2, 1)]:
+        o, lse, _ = _run(lib, q, k, v, B=len(lens), Hq=Hq, Hkv=Hkv, N=T, d=d, scale=0.6,
+                         causal=causal, window_left=left, window_right=right, cu_seqlens=cu)
+        for b, L in enumerate(lens):
+            a = cu[b]
+            ob, lb, _ = _run(lib, q[a:a + L].unsqueeze(0).contiguous(),
+                             k[a:a + L].unsqueeze(0).contiguous(),
+                             v[a:a + L].unsqueeze(0).contiguous(), B=1, Hq=Hq, Hkv=Hkv, N=L,
+                             d=d, scale=0.6, causal=causal, window_left=left, window_right=right)
+            assert np.array_equal(o[a:a + L], ob)
+            assert np.array_equal(lse[:, a:a + L], lb[0])
+
+
+def pin_gqa_equals_repeated(lib):
+    rng = np.random.default_rng(20)
+    B, N, Hq, Hkv, d = 2, 19, 6, 2, 8
+    q = _bf16(rng.standard_normal((B, N, Hq, d)))
+    k = _bf16(rng.standard_normal((B, N, Hkv, d)))
+    v = _bf16(rng.standard_normal((B, N, Hkv, d)))
+    o, lse, _ = _run(lib, q, k, v, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=0.5, causal=True)
+    kr = torch.repeat_interleave(k, Hq // Hkv, dim=2).contiguous()
+    vr = torch.repeat_interleave(v, Hq // Hkv, dim=2).contiguous()
+    o2, lse2, _ = _run(lib, q, kr, vr, B=B, Hq=Hq, Hkv=Hq, N=N, d=d, scale=0.5, causal=True)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+# --------------------------------------------------------------------------
+# independent library routine
+# --------------------------------------------------------------------------
+def _band_mask(N, causal, left, right):
+    """Visible-key matrix from torch.triu/torch.tril, as the page's recipe builds
+    its causal mask with torch.triu(ones, 1)."""
+    ones = torch.ones(N, N, dtype=torch.bool)
+    if causal:
+        right = 0
+    allowed = ones.clone()
+    if right >= 0:
+        allowed &= ~torch.triu(ones, diagonal=right + 1)
+    if left >= 0:
+        allowed &= ~torch.tril(ones, diagonal=-left - 1)
+    return allowed
+
+
+def pin_torch_sdpa(lib):
+    import torch.nn.functional as F
+    rng = np.random.default_rng(21)
+    cases = [
+        # B, N, Hq, Hkv, d, causal, left, right, scale
+        (2, 45, 4, 4, 32, False, -1, -1, 32 ** -0.5),
+        (1, 70, 4, 2, 64, True, -1, -1, 64 ** -0.5),
+        (2, 33, 6, 3, 16, True, 7, 0, 0.3),
+        (1, 50, 2, 1, 8, False, 3, 9, 1.1),
+    ]
+    for (B, N, Hq, Hkv, d, causal, left, right, scale) in cases:
+        q = _bf16(rng.standard_normal((B, N, Hq, d)))
+        k = _bf16(rng.standard_normal((B, N, Hkv, d)))
+        v = _bf16(rng.standard_normal((B, N, Hkv, d)))
+        o, lse, _ = _run(lib, q, k, v, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=scale,
+                         causal=causal, window_left=left, window_right=right)
+        o = o.reshape(B, N, Hq, d)
+        g = Hq // Hkv
+        qt = q.to(torch.float64).transpose(1, 2)  # [B,H,N,d]
+        kt = torch.repeat_interleave(k.to(torch.float64), g, dim=2).transpose(1, 2)
+        vt = torch.repeat_interleave(v.to(torch.float64), g, dim=2).transpose(1, 2)
+        mask = _band_mask(N, causal, left, right)
+        ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+        ref = ref.transpose(1, 2).numpy()
+        assert np.abs(o - ref).max() <= 1e-12, np.abs(o - ref).max()
+        scores = (qt @ kt.transpose(-1, -2)) * scale
+        ref_lse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1).numpy()
+        assert np.abs(lse - ref_lse).max() <= 1e-12
+
+
+def pin_rows_mode_matches_full(lib):
+    """The sampled-row entry (used at full workload sizes) equals the full run."""
+    rng = np.random.default_rng(22)
+    lens = [9, 30, 2]
+    cu = W.cumulative(lens)
+    T, Hq, Hkv, d = cu[-1], 4, 1, 16
+    q = _bf16(rng.standard_normal((T, Hq, d)))
+    k = _bf16(rng.standard_normal((T, Hkv, d)))
+    v = _bf16(rng.standard_normal((T, Hkv, d)))
+    o, lse, nv = _run(lib, q, k, v, B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=0.5, causal=True,
+                      window_left=6, cu_seqlens=cu)
+    rows = np.array([[1, 2, 17], [0, 0, 0], [2, 3, 1], [1, 1, 29]], dtype=np.int64)
+    o2, lse2, nv2 = _run(lib, q, k, v, B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=0.5, causal=True,
+                         window_left=6, cu_seqlens=cu, rows=rows)
+    for r, (b, h, i) in enumerate(rows):
+        t = cu[b] + i
+        assert np.array_equal(o2[r], o[t, h])
+        assert lse2[r] == lse[h, t] and nv2[r] == nv[h, t]
+
+
+ALL_PINS = [
+    pin_worked_example,
+    pin_uniform_scores,
+    pin_uniform_scores_packed,
+    pin_two_keys,
+    pin_hard_limit,
+    pin_single_key_and_row0,
+    pin_constant_v_and_row_sums,
+    pin_key_permutation,
+    pin_window_equals_causal,
+    pin_packed_equals_separate,
+    pin_gqa_equals_repeated,
+    pin_torch_sdpa,
+    pin_rows_mode_matches_full,
+]

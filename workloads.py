@@ -1,0 +1,128 @@
+"""Seeded synthetic inputs, shared by the CUDA path's tests/bench and the oracle.
+
+This module holds no attention arithmetic: only shapes, seeds and random draws.
+Both sides receive the very same host bytes from it.
+
+Recipe (one fixed rule for every workload):
+  torch.manual_seed(seed); q, k, v = torch.randn(shape, float32) drawn in that
+  order on the CPU, each then rounded to bfloat16.
+  Dense shapes are [B, N, H, d] ("Flash Attention" skill page (skillmd.com),
+  Workflow 2: input [batch_size, seq_len, num_heads, head_dim]); packed
+  variable-length shapes are [tokens, H, d] with int32 cumulative boundaries.
+  The pages time normal-random bf16/fp16 tensors of this kind ("FlashAttention"
+  explainer page, "A simple benchmark script"); no dataset is involved.
+
+The five named workloads are the ones the benchmark and the parity tests use.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+
+@dataclass
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int  # dense: sequence length; packed: total tokens
+    d: int
+    causal: bool
+    window_left: int
+    window_right: int
+    seed: int
+    cu_seqlens: Optional[List[int]] = None
+    max_seqlen: int = 0
+    scale: float = field(default=0.0)
+
+    def __post_init__(self):
+        if self.scale == 0.0:
+            self.scale = default_scale(self.d)
+        if self.max_seqlen == 0:
+            if self.cu_seqlens is None:
+                self.max_seqlen = self.N
+            else:
+                self.max_seqlen = max(b - a for a, b in zip(self.cu_seqlens[:-1], self.cu_seqlens[1:]))
+
+    @property
+    def tokens(self) -> int:
+        return self.cu_seqlens[-1] if self.cu_seqlens is not None else self.B * self.N
+
+    @property
+    def packed(self) -> bool:
+        return self.cu_seqlens is not None
+
+
+def default_scale(d: int) -> float:
+    """1/sqrt(d) as the fp32 value that is passed to both sides."""
+    return float(np.float32(1.0 / math.sqrt(d)))
+
+
+def packed_lengths(seed: int = 4, total: int = 65536, lo: int = 128, hi: int = 4096) -> List[int]:
+    """Sequence lengths drawn uniform in [lo, hi] until `total` tokens; the last
+    one is truncated so the lengths sum to exactly `total`."""
+    rng = np.random.default_rng(seed)
+    out: List[int] = []
+    acc = 0
+    while acc < total:
+        L = int(rng.integers(lo, hi + 1))
+        L = min(L, total - acc)
+        out.append(L)
+        acc += L
+    return out
+
+
+def cumulative(lengths: List[int]) -> List[int]:
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + int(L))
+    return cu
+
+
+def workload(cfg: int) -> Workload:
+    """The five named workloads (1 is small enough for a full oracle run)."""
+    if cfg == 1:
+        return Workload("noncausal_b1_h2_n256_d64", 1, 2, 2, 256, 64, False, -1, -1, 0)
+    if cfg == 2:
+        return Workload("causal_mha_b4_h16_n2048_d128", 4, 16, 16, 2048, 128, True, -1, -1, 1)
+    if cfg == 3:
+        return Workload("causal_gqa_b2_hq32_hkv8_n8192_d128", 2, 32, 8, 8192, 128, True, -1, -1, 2)
+    if cfg == 4:
+        return Workload("swa_b1_h32_n16384_d128_left4096", 1, 32, 32, 16384, 128, True, 4096, 0, 3)
+    if cfg == 5:
+        cu = cumulative(packed_lengths(4))
+        return Workload("varlen_causal_t65536_hq32_hkv8_d128", len(cu) - 1, 32, 8, cu[-1], 128,
+                        True, -1, -1, 4, cu_seqlens=cu)
+    raise ValueError(f"unknown workload {cfg}")
+
+
+def draw_qkv(shape_q, shape_kv, seed: int):
+    """q, k, v as CPU bf16 tensors (fp32 normal draws rounded to bf16)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn(shape_q, dtype=torch.float32, generator=g).to(torch.bfloat16)
+    k = torch.randn(shape_kv, dtype=torch.float32, generator=g).to(torch.bfloat16)
+    v = torch.randn(shape_kv, dtype=torch.float32, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def inputs(w: Workload):
+    """(q, k, v) CPU bf16 tensors for a workload; packed workloads are [T, H, d]."""
+    if w.packed:
+        return draw_qkv((w.tokens, w.Hq, w.d), (w.tokens, w.Hkv, w.d), w.seed)
+    return draw_qkv((w.B, w.N, w.Hq, w.d), (w.B, w.N, w.Hkv, w.d), w.seed)
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """View a CPU bf16 tensor as its uint16 bit patterns (no copy of values)."""
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def from_bits(a: np.ndarray) -> torch.Tensor:
+    """Inverse of bf16_bits."""
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
