@@ -1,0 +1,420 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused attention forward (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5] [--impl reference]
+
+A step is one call of the fused forward (the whole hot path) over one batch of
+the workload.  The default workload is the causal grouped-query forward at
+N = 8192 (B=2, Hq=32, Hkv=8, d=128), the first pure causal d = 128 case with
+N >= 8192.  Inputs are seeded synthetic normal bf16 tensors (workloads.py).
+
+Metric: TFLOP/s = 4 * d * (visible query/key pairs) * Hq / time, counting only
+unmasked pairs (diagonal included).  Device time comes from CUDA events on the
+launching stream; L2 is flushed between timed steps (outside the events).
+`e2e` repeats the measurement through the host-buffer C entry point
+(attn_fwd_host) with pinned host buffers: host->device copies of q, k, v, the
+kernel and device->host copies of o and lse are all inside the timed region.
+
+With N > 1 (torchrun, one process per GPU) every rank runs the same workload on
+its own GPU (independent replicas, weak scaling); the time is the max over
+ranks and the value is all ranks' FLOPs over that time.  There is no
+collective on the data path.
+
+--impl reference times the CPU oracle (fp64, all host cores) on bounded
+samples of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s (bf16, causal, d=128) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+SPEC_BF16_TFLOPS = 2250.0   # NVIDIA datasheet dense bf16, for context
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["exact_attention_142_b200/csrc/attn_fwd_kernel.cuh",
+                  "exact_attention_142_b200/csrc/ptx.cuh",
+                  "exact_attention_142_b200/csrc/attn_api.cu"]
+
+
+def visible_pairs(w: W.Workload) -> int:
+    """Number of visible (query, key) pairs per head, summed over sequences."""
+    right = 0 if w.causal else w.window_right
+    left = w.window_left
+    lengths = ([b - a for a, b in zip(w.cu_seqlens[:-1], w.cu_seqlens[1:])] if w.packed
+               else [w.N] * w.B)
+    total = 0
+    for L in lengths:
+        i = np.arange(L, dtype=np.int64)
+        lo = np.zeros(L, np.int64) if left < 0 else np.maximum(0, i - left)
+        hi = np.full(L, L - 1, np.int64) if right < 0 else np.minimum(L - 1, i + right)
+        total += int((hi - lo + 1).sum())
+    return total
+
+
+def flops_of(w: W.Workload) -> float:
+    return 4.0 * w.d * visible_pairs(w) * w.Hq
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {}, "fallback"
+
+
+def kernel_sources_digest() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload_name}_traffic.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_sources_digest():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.sw_power_cap,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._thr = threading.Thread(target=self._read, daemon=True)
+            self._thr.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sel = [l for (t, l) in self.lines if self.t0 is None or (self.t0 <= t <= (self.t1 or t) + 0.06)]
+        if not sel:
+            sel = [l for (_, l) in self.lines]
+        sm, mx, pw = [], [], []
+        reasons = set()
+        names = ["sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+        for l in sel:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------
+def run_cuda(args, w: W.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_142_b200 as ea
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    q, k, v = W.inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(qd)
+    if w.packed:
+        cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=dev)
+        lse = torch.empty((w.Hq, w.tokens), dtype=torch.float32, device=dev)
+    else:
+        cu = None
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_fwd(qd, kd, vd, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                    w.window_left, w.window_right, cu, w.max_seqlen, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported a timeout during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    for i in range(args.steps):
+        flush.zero_()  # evict L2 (outside the timed events)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.mark_end()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kernel_ms = sum(times) / len(times)
+    status = ea.attn_device_status()
+    if status != ea.ATTN_OK:
+        raise RuntimeError(f"device status {status} during the timed region")
+
+    # end to end through the host-buffer entry point
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+    cuh = torch.tensor(w.cu_seqlens, dtype=torch.int32) if w.packed else None
+    nbytes = ea.attn_fwd_host_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d, w.packed)
+    del qd, kd, vd, o
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        ea.attn_fwd_host(qh, kh, vh, oh, lh, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                         w.window_left, w.window_right, cuh, w.max_seqlen, ws, nbytes, stream)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(3, min(args.steps, 20))
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(e_steps):
+        es[i].record(stream)
+        e2e_step()
+        ee[i].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es, ee)) / e_steps
+    h2d = (q.numel() + k.numel() + v.numel()) * 2 + (4 * len(w.cu_seqlens) if w.packed else 0)
+    d2h = oh.numel() * 2 + lh.numel() * 4
+
+    clocks = sampler.stop() if sampler else None
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([kernel_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        kernel_ms, e2e_ms = float(t[0]), float(t[1])
+    return kernel_ms, e2e_ms, h2d, d2h, clocks
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU) timing
+# ---------------------------------------------------------------------------
+def oracle_sample(w: W.Workload, q, k, v, nrows: int, seed: int):
+    """Time the oracle on `nrows` (sequence, head, row) triples drawn uniformly
+    from the workload; returns (seconds, flops of those rows, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    lengths = ([b - a for a, b in zip(w.cu_seqlens[:-1], w.cu_seqlens[1:])] if w.packed
+               else [w.N] * w.B)
+    cum = np.cumsum([0] + lengths)
+    flat = rng.integers(0, cum[-1], size=nrows)
+    b = np.searchsorted(cum, flat, side="right") - 1
+    i = flat - cum[b]
+    h = rng.integers(0, w.Hq, size=nrows)
+    rows = np.stack([b, h, i], axis=1).astype(np.int64)
+    qb, kb, vb = W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v)
+    t0 = time.perf_counter()
+    _, _, nvis = oracle.attn_fwd(qb, kb, vb, B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d,
+                                 scale=w.scale, causal=w.causal, window_left=w.window_left,
+                                 window_right=w.window_right, cu_seqlens=w.cu_seqlens, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, 4.0 * w.d * float(nvis.sum()), oracle.num_threads()
+
+
+def calibrate_rows(w, q, k, v, target_s: float) -> int:
+    rows = 64
+    dt, _, _ = oracle_sample(w, q, k, v, rows, seed=1)
+    while dt < 0.5 and rows < (1 << 22):
+        rows *= 4
+        dt, _, _ = oracle_sample(w, q, k, v, rows, seed=1)
+    return max(16, int(rows * target_s / max(dt, 1e-6)))
+
+
+def cpu_baseline(w: W.Workload, target_s: float = 12.0):
+    q, k, v = W.inputs(w)
+    rows = calibrate_rows(w, q, k, v, target_s)
+    dt, fl, thr = oracle_sample(w, q, k, v, rows, seed=2)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{rows} query rows drawn uniformly over (sequence, head, row) of the "
+                      f"workload, fp64 oracle, {dt:.1f} s on {thr} threads"}
+
+
+def run_reference(args, w: W.Workload):
+    """The oracle as the reference arm: K timed steps, each a bounded sample."""
+    q, k, v = W.inputs(w)
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    rows = calibrate_rows(w, q, k, v, min(budget_s, 30.0))
+    for i in range(args.warmup):
+        oracle_sample(w, q, k, v, rows, seed=10 + i)
+    tot_t, tot_f, thr = 0.0, 0.0, 1
+    for i in range(args.steps):
+        dt, fl, thr = oracle_sample(w, q, k, v, rows, seed=1000 + i)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, args.gpus), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"{rows} query rows per step, drawn uniformly over "
+                                   f"(sequence, head, row); fp64 oracle on {thr} threads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def config_dict(w: W.Workload, n_gpus: int):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+            "N": w.N if not w.packed else None, "tokens": w.tokens, "d": w.d,
+            "causal": w.causal, "window": [w.window_left, w.window_right],
+            "packed_sequences": len(w.cu_seqlens) - 1 if w.packed else None,
+            "flop_per_step": flops_of(w), "l2": "flushed between timed steps",
+            "parallelism": f"replicas x{n_gpus} (no collective)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = W.workload(args.workload)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        kernel_ms, e2e_ms, h2d, d2h, clocks = run_cuda(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.barrier()
+    if rank == 0:
+        fl = flops_of(w)
+        value = fl * world / (kernel_ms * 1e-3) / 1e12
+        achieved = fl / (kernel_ms * 1e-3) / 1e12
+        peaks, src = measured_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        sustained = float(peaks.get("bf16_tflops_sustained", 0.0)) or None
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": kernel_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal bf16 Q, K, V)",
+            "config": config_dict(w, world),
+            "e2e": {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                         "peak_source": f"{src} bf16_tflops (burst, cuBLAS)" if src == "measured"
+                         else "fallback 1590 TF/s",
+                         "frac_of_sustained": (achieved / sustained) if sustained else None,
+                         "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
+                         "kernel": "attn_fwd_sm100<128,5>" if w.d == 128 else "attn_fwd_sm100<64,8>"},
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,131 @@
+"""ctypes binding of the C ABI in include/attn.h (argument marshalling only).
+
+Every entry point keeps the C name.  Tensors may be passed as torch tensors
+(their data pointer is used) or as raw integer addresses; streams as
+torch.cuda.Stream, a raw handle, or None for torch's current stream.  All
+computation happens in the CUDA library; there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b200.so")
+_lib = None
+_lock = threading.Lock()
+
+ATTN_OK = 0
+ATTN_ERR_NULL = -1
+ATTN_ERR_SHAPE = -2
+ATTN_ERR_WINDOW = -3
+ATTN_ERR_UNSUPPORTED = -4
+ATTN_ERR_ALIGN = -5
+ATTN_ERR_CUDA = -6
+ATTN_ERR_SCALE = -7
+ATTN_ERR_WORKSPACE = -8
+ATTN_ERR_DEVICE_TIMEOUT = -9
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str = "attn_fwd"):
+        self.status = status
+        super().__init__(f"{what} failed: {attn_status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library; raise loudly if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {_LIB_PATH} is missing; build it with "
+                "`python -m exact_attention_142_b200.build` (there is no fallback)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.attn_fwd.restype = I
+        lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P]
+        lib.attn_fwd_host.restype = I
+        lib.attn_fwd_host.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P, S, P]
+        lib.attn_fwd_host_workspace_bytes.restype = S
+        lib.attn_fwd_host_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        lib.attn_status_string.argtypes = [I]
+        lib.attn_device_status.restype = I
+        lib.attn_device_status.argtypes = []
+        lib.attn_selftest_bounded_wait.restype = I
+        lib.attn_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
+        _lib = lib
+        return lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr() if x.numel() > 0 else None
+    if hasattr(x, "ctypes"):  # numpy array
+        return x.ctypes.data
+    raise TypeError(f"cannot take a pointer of {type(x)}")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window_left=-1,
+             window_right=-1, cu_seqlens=None, max_seqlen=0, stream=None, check=True) -> int:
+    """Enqueue the fused forward on device buffers (see include/attn.h)."""
+    lib = load_library()
+    rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq), int(Hkv),
+                      int(N), int(d), float(scale), int(bool(causal)), int(window_left),
+                      int(window_right), _ptr(cu_seqlens), int(max_seqlen), _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc)
+    return rc
+
+
+def attn_fwd_host_workspace_bytes(B, Hq, Hkv, N, d, packed) -> int:
+    return int(load_library().attn_fwd_host_workspace_bytes(int(B), int(Hq), int(Hkv), int(N),
+                                                            int(d), int(bool(packed))))
+
+
+def attn_fwd_host(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window_left=-1,
+                  window_right=-1, cu_seqlens=None, max_seqlen=0, workspace=None,
+                  workspace_bytes=0, stream=None, check=True) -> int:
+    """Same operation on host buffers; copies run on `stream` (see include/attn.h)."""
+    lib = load_library()
+    rc = lib.attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq),
+                           int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
+                           int(window_left), int(window_right), _ptr(cu_seqlens), int(max_seqlen),
+                           _ptr(workspace), int(workspace_bytes), _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_host")
+    return rc
+
+
+def attn_status_string(status: int) -> str:
+    return load_library().attn_status_string(int(status)).decode()
+
+
+def attn_device_status() -> int:
+    return int(load_library().attn_device_status())
+
+
+def attn_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    return int(load_library().attn_selftest_bounded_wait(int(limit_ns), _stream(stream)))

@@ -1,0 +1,269 @@
+// attn_api.cu -- C ABI of the fused attention forward (declared in attn.h):
+// argument validation, TMA tensor-map encoding, launch configuration, the
+// host-buffer variant, and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace {
+
+using attn::FwdParams;
+
+constexpr int kStages128 = 5;  // K/V ring depth at d = 128 (32 KB per slot)
+constexpr int kStages64 = 8;   // at d = 64 (16 KB per slot)
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
+                cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// [rows, cols] bf16, row stride cols * 2 bytes; boxes of 128 rows x 64 columns
+// (128 bytes) with 128-byte swizzling.  Rows past the end read as zero.
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estride[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+    int checked = 0;  // 1 = supported, -1 = unsupported
+    bool smem_set64 = false, smem_set128 = false;
+};
+DeviceState g_devices[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Checks the current device (sm_100) and prepares the kernels' shared-memory
+// limit once per device.
+int prepare_device(int d) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceState& st = g_devices[dev];
+    if (st.checked == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        st.checked = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    if (st.checked < 0) return ATTN_ERR_UNSUPPORTED;
+    if (d == 128 && !st.smem_set128) {
+        if (cudaFuncSetAttribute(attn::attn_fwd_sm100<128, kStages128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)attn::SmemLayout<128, kStages128>::kDynamicBytes) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        st.smem_set128 = true;
+    }
+    if (d == 64 && !st.smem_set64) {
+        if (cudaFuncSetAttribute(attn::attn_fwd_sm100<64, kStages64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)attn::SmemLayout<64, kStages64>::kDynamicBytes) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        st.smem_set64 = true;
+    }
+    return ATTN_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Host-side checks shared by both entry points.  `tokens` is set to the
+// number of packed tokens (B * N in dense mode).
+int validate(const void* q, const void* k, const void* v, const void* o, const float* lse, int B,
+             int Hq, int Hkv, int N, int d, float scale, int window_left, int window_right,
+             bool packed, int max_seqlen, long long* tokens) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N < 0) return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+    if (window_left < -1 || window_right < -1) return ATTN_ERR_WINDOW;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_SCALE;
+    const long long t = packed ? (long long)N : (long long)B * N;
+    if (t > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+    if ((long long)Hq * d > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+    if (packed && N > 0 && max_seqlen <= 0) return ATTN_ERR_SHAPE;
+    *tokens = t;
+    if (t == 0) return ATTN_OK;
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return ATTN_ERR_ALIGN;
+    return ATTN_OK;
+}
+
+template <int D, int STAGES>
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+           long long units, cudaStream_t stream) {
+    attn::attn_fwd_sm100<D, STAGES><<<(unsigned)units, attn::kThreads,
+                                       attn::SmemLayout<D, STAGES>::kDynamicBytes, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                        int window_right, const int32_t* cu_seqlens, int max_seqlen,
+                        struct CUstream_st* stream) {
+    const bool packed = cu_seqlens != nullptr;
+    long long tokens = 0;
+    int rc = validate(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, window_left, window_right, packed,
+                      max_seqlen, &tokens);
+    if (rc != ATTN_OK) return rc;
+    if (tokens == 0) return ATTN_OK;
+    rc = prepare_device(d);
+    if (rc != ATTN_OK) return rc;
+
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, (uint64_t)tokens, (uint64_t)Hq * d) ||
+        !make_map(&mk, k, (uint64_t)tokens, (uint64_t)Hkv * d) ||
+        !make_map(&mv, v, (uint64_t)tokens, (uint64_t)Hkv * d))
+        return ATTN_ERR_CUDA;
+
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens = cu_seqlens;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.group = Hq / Hkv;
+    p.left = window_left;
+    p.right = causal ? 0 : window_right;
+    p.pair_mode = (p.group % 2 == 0) ? attn::kPairHeads : attn::kPairRows;
+    const int max_len = packed ? (max_seqlen < N ? max_seqlen : N) : N;
+    p.n_row_blocks = (max_len + attn::kBM - 1) / attn::kBM;
+    p.scale = scale;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+    p.wait_limit_ns = kWaitLimitNs;
+
+    const long long units = p.pair_mode == attn::kPairHeads
+                                ? (long long)p.n_row_blocks * B * (Hq / 2)
+                                : (long long)((p.n_row_blocks + 1) / 2) * B * Hq;
+    if (units <= 0) return ATTN_OK;
+    if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return d == 128 ? launch<128, kStages128>(mq, mk, mv, p, units, s)
+                    : launch<64, kStages64>(mq, mk, mv, p, units, s);
+}
+
+extern "C" size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int packed) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0) return 0;
+    const size_t tokens = packed ? (size_t)N : (size_t)B * (size_t)N;
+    size_t total = 0;
+    total += round256(tokens * Hq * d * 2);       // q
+    total += 2 * round256(tokens * Hkv * d * 2);  // k, v
+    total += round256(tokens * Hq * d * 2);       // o
+    total += round256(tokens * Hq * 4);           // lse
+    if (packed) total += round256((size_t)(B + 1) * 4);
+    return total;
+}
+
+extern "C" int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                             int window_left, int window_right, const int32_t* cu_seqlens,
+                             int max_seqlen, void* workspace, size_t workspace_bytes,
+                             struct CUstream_st* stream) {
+    const bool packed = cu_seqlens != nullptr;
+    if (packed && max_seqlen <= 0) {  // derive it from the host boundaries
+        max_seqlen = 0;
+        for (int b = 0; b < B; ++b) {
+            const int L = cu_seqlens[b + 1] - cu_seqlens[b];
+            if (L > max_seqlen) max_seqlen = L;
+        }
+    }
+    long long tokens = 0;
+    int rc = validate(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, window_left, window_right, packed,
+                      max_seqlen, &tokens);
+    if (rc != ATTN_OK) return rc;
+    if (tokens == 0) return ATTN_OK;
+    const size_t need = attn_fwd_host_workspace_bytes(B, Hq, Hkv, N, d, packed ? 1 : 0);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
+
+    const size_t bq = (size_t)tokens * Hq * d * 2, bkv = (size_t)tokens * Hkv * d * 2;
+    const size_t bl = (size_t)tokens * Hq * 4;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* dq = ws;
+    uint8_t* dk = dq + round256(bq);
+    uint8_t* dv = dk + round256(bkv);
+    uint8_t* dout = dv + round256(bkv);
+    uint8_t* dlse = dout + round256(bq);
+    int32_t* dcu = packed ? reinterpret_cast<int32_t*>(dlse + round256(bl)) : nullptr;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(dq, q, bq, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, bkv, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, bkv, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (packed && cudaMemcpyAsync(dcu, cu_seqlens, (size_t)(B + 1) * 4, cudaMemcpyHostToDevice, s) !=
+                      cudaSuccess)
+        return ATTN_ERR_CUDA;
+    rc = attn_fwd(dq, dk, dv, dout, reinterpret_cast<float*>(dlse), B, Hq, Hkv, N, d, scale, causal,
+                  window_left, window_right, dcu, max_seqlen, stream);
+    if (rc != ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o, dout, bq, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse, dlse, bl, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+extern "C" const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_NULL: return "a required pointer is NULL";
+        case ATTN_ERR_SHAPE: return "invalid sizes (B, Hq, Hkv, N, max_seqlen or Hq % Hkv)";
+        case ATTN_ERR_WINDOW: return "window_left / window_right must be -1 or >= 0";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported head dimension (64, 128) or device (sm_100)";
+        case ATTN_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
+        case ATTN_ERR_CUDA: return "a CUDA runtime or driver call failed";
+        case ATTN_ERR_SCALE: return "scale must be finite and > 0";
+        case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out; outputs are undefined";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int attn_device_status(void) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return v;
+}
+
+extern "C" int attn_selftest_bounded_wait(uint64_t limit_ns, struct CUstream_st* stream) {
+    if (limit_ns < 1000ull) limit_ns = 1000ull;
+    if (limit_ns > 2000000000ull) limit_ns = 2000000000ull;
+    attn::selftest_bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)limit_ns);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}

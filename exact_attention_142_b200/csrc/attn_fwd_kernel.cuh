@@ -1,0 +1,608 @@
+// attn_fwd_kernel.cuh -- fused exact attention forward for sm_100a.
+//
+// One CTA owns two 128-row query tiles that read the same key/value head and
+// streams 128-key blocks of K and V through a shared-memory ring:
+//
+//   warps 0-3  softmax for query tile 0 (one thread per query row)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    producer: TMA loads of Q (once) and of the K/V ring
+//   warp  9    MMA issuer: tcgen05 S = Q K^T (both operands in shared memory)
+//              and O += P V (P read from tensor memory)
+//   warps 10-11 spare (complete the third warpgroup)
+// Registers move from the third warpgroup to the two softmax warpgroups with
+// setmaxnreg (the whole score row of a query lives in one thread).
+//
+// Tensor memory (512 columns, fp32): S0 [0,128), S1 [128,256), O0 [256,384),
+// O1 [384,512).  Each softmax thread loads its whole score row, writes the
+// bf16 weights P back into the upper half of the same S columns, and the PV
+// product reads them from there.
+//
+// Algorithm ("FlashAttention", ozercemkelahmet.com/tools/flashattention,
+// "How it works"): Step 1 tiles along the sequence, Step 2 scores per tile on
+// chip, Step 3 online softmax with a running maximum and running sum whose old
+// values are rescaled when the maximum grows, Step 4 the output accumulated
+// with the same correction and divided by the final sum once, Step 5 the
+// per-row log-sum-exp saved, Step 6 whole key blocks outside the causal or
+// sliding-window band skipped and the boundary blocks masked element-wise,
+// Step 7 the work spread over (query block, batch, head), Step 8 16-bit
+// operands with fp32 accumulation and fp32 statistics.
+//
+// The running maximum is allowed to lag the true maximum by up to 2^8 in the
+// exponent (the correction of O is skipped until the growth exceeds that).
+// This stays exact: every weight and the sum use the same reference maximum,
+// so the final division cancels it.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "attn.h"
+#include "ptx.cuh"
+
+namespace attn {
+
+// Device status word (one per device); see attn_device_status().  All kernels
+// are compiled in one translation unit, which owns this definition.
+__device__ int g_attn_status = 0;
+
+constexpr int kBM = 128;        // query rows per tile
+constexpr int kBN = 128;        // keys per block
+constexpr int kThreads = 384;   // 8 softmax warps + producer + MMA + 2 spare
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO0 = 256;
+constexpr uint32_t kPOffset = 64;      // P columns inside an S region
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLn2 = 0.693147180559945309f;
+// Register split after launch (384 threads x 168 = 64512 registers):
+// 128 x (216 + 216 + 72) = 64512.
+constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsOther = 72;
+
+enum : int { kPairHeads = 0, kPairRows = 1 };
+
+struct FwdParams {
+    void* o;
+    float* lse;
+    const int32_t* cu_seqlens;  // nullptr in dense mode
+    int B, Hq, Hkv;
+    int N;             // dense: sequence length; packed: total tokens
+    int group;         // Hq / Hkv
+    int left, right;   // -1 = unlimited; causal is already folded into right = 0
+    int pair_mode;     // kPairHeads: heads (2p, 2p+1) of one row block
+                       // kPairRows : row blocks (2p, 2p+1) of one head
+    int n_row_blocks;  // ceil(max sequence length / 128)
+    float scale_log2;  // scale * log2(e)
+    float scale;
+    unsigned long long wait_limit_ns;
+};
+
+template <int D, int STAGES>
+struct SmemLayout {
+    static constexpr uint32_t kTileBytes = kBM * D * 2;  // one Q, K or V tile (bf16)
+    static constexpr uint32_t kBoxBytes = 128 * 128;     // one TMA box: 128 rows x 128 bytes
+    static constexpr uint32_t kQ0 = 0;
+    static constexpr uint32_t kQ1 = kTileBytes;
+    static constexpr uint32_t kKV = 2 * kTileBytes;
+    static constexpr uint32_t kBar = kKV + STAGES * kTileBytes;
+    // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final
+    static constexpr uint32_t kNumBars = 8 + 2 * STAGES;
+    static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem address, abort flag
+    static constexpr uint32_t kBytes = kMisc + 16;
+    static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // room to align the base to 1 KB
+
+    static __device__ __forceinline__ uint32_t bar_q(uint32_t base) { return base + kBar; }
+    static __device__ __forceinline__ uint32_t bar_kv_full(uint32_t base, int s) {
+        return base + kBar + 8u * (1 + s);
+    }
+    static __device__ __forceinline__ uint32_t bar_kv_empty(uint32_t base, int s) {
+        return base + kBar + 8u * (1 + STAGES + s);
+    }
+    static __device__ __forceinline__ uint32_t bar_s_full(uint32_t base, int x) {
+        return base + kBar + 8u * (1 + 2 * STAGES + x);
+    }
+    static __device__ __forceinline__ uint32_t bar_p_ready(uint32_t base, int x) {
+        return base + kBar + 8u * (3 + 2 * STAGES + x);
+    }
+    static __device__ __forceinline__ uint32_t bar_o_done(uint32_t base, int x) {
+        return base + kBar + 8u * (5 + 2 * STAGES + x);
+    }
+    static __device__ __forceinline__ uint32_t bar_mma_final(uint32_t base) {
+        return base + kBar + 8u * (7 + 2 * STAGES);
+    }
+};
+
+// Wait for an mbarrier phase with a time limit.  On expiry the block-wide
+// abort flag is raised and the device status word records the timeout; once
+// the flag is up every other bounded wait of the block returns at once.
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long limit_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (ptx::global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicCAS(&g_attn_status, 0, ATTN_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Teardown wait for work already in flight (TMA copies, MMAs): ignores the
+// abort flag but is still bounded.
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity,
+                                           unsigned long long limit_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::global_timer_ns() - t0 > limit_ns) {
+            atomicCAS(&g_attn_status, 0, ATTN_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// The two query tiles of one CTA and the key blocks each of them needs.
+struct TilePair {
+    int b, start, len, g;
+    int h[2];
+    int r0[2];
+    int lo[2], hi[2];  // key-block range [lo, hi); empty when the tile is inactive
+    bool active[2];
+    int ulo, uhi;      // union of the two ranges
+};
+
+__device__ __forceinline__ TilePair decode_pair(int u, const FwdParams& p) {
+    TilePair w;
+    int t[2];
+    if (p.pair_mode == kPairHeads) {
+        const int hp_count = p.Hq / 2;
+        const int per_t = p.B * hp_count;
+        const int tb = p.n_row_blocks - 1 - u / per_t;  // heaviest (latest) rows first
+        const int rem = u % per_t;
+        w.b = rem / hp_count;
+        const int hp = rem % hp_count;
+        w.h[0] = 2 * hp;
+        w.h[1] = 2 * hp + 1;
+        t[0] = t[1] = tb;
+    } else {
+        const int np = (p.n_row_blocks + 1) / 2;
+        const int per_t = p.B * p.Hq;
+        const int tp = np - 1 - u / per_t;
+        const int rem = u % per_t;
+        w.b = rem / p.Hq;
+        w.h[0] = w.h[1] = rem % p.Hq;
+        t[0] = 2 * tp;
+        t[1] = 2 * tp + 1;
+    }
+    if (p.cu_seqlens) {
+        w.start = p.cu_seqlens[w.b];
+        w.len = p.cu_seqlens[w.b + 1] - w.start;
+    } else {
+        w.start = w.b * p.N;
+        w.len = p.N;
+    }
+    w.g = w.h[0] / p.group;
+    w.ulo = 0x7fffffff;
+    w.uhi = 0;
+    for (int x = 0; x < 2; ++x) {
+        w.r0[x] = t[x] * kBM;
+        w.active[x] = w.r0[x] < w.len;
+        if (w.active[x]) {
+            const long long kv_lo = p.left >= 0 ? (long long)w.r0[x] - p.left : 0;
+            const long long kv_hi =
+                p.right >= 0 ? (long long)w.r0[x] + kBM + p.right : (long long)w.len;
+            const long long lo_c = kv_lo < 0 ? 0 : kv_lo;
+            const long long hi_c = kv_hi > w.len ? w.len : kv_hi;
+            w.lo[x] = (int)(lo_c / kBN);
+            w.hi[x] = (int)((hi_c + kBN - 1) / kBN);
+            if (w.lo[x] < w.ulo) w.ulo = w.lo[x];
+            if (w.hi[x] > w.uhi) w.uhi = w.hi[x];
+        } else {
+            w.lo[x] = w.hi[x] = 0;
+        }
+    }
+    if (w.uhi <= w.ulo) w.ulo = w.uhi = 0;
+    return w;
+}
+
+__device__ __forceinline__ bool tile_active_at(const TilePair& w, int x, int j) {
+    return w.active[x] && j >= w.lo[x] && j < w.hi[x];
+}
+
+// ---------------------------------------------------------------- producer
+template <int D, int STAGES>
+__device__ __forceinline__ void producer_role(const TilePair& w, const FwdParams& p,
+                                              const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                              const CUtensorMap* tm_v, uint32_t sbase,
+                                              volatile int* abort_flag) {
+    using L = SmemLayout<D, STAGES>;
+    constexpr int kBoxes = D / 64;
+    const uint64_t pol_q = ptx::policy_evict_first();
+    const uint64_t pol_kv = ptx::policy_evict_last();
+
+    ptx::mbar_arrive_expect_tx(L::bar_q(sbase), 2 * L::kTileBytes);
+    for (int x = 0; x < 2; ++x) {
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx)
+            ptx::tma_load_2d(sbase + (x ? L::kQ1 : L::kQ0) + bx * L::kBoxBytes, tm_q,
+                             L::bar_q(sbase), w.h[x] * D + bx * 64, w.start + w.r0[x], pol_q);
+    }
+
+    int issued = 0;
+    bool ok = true;
+    for (int j = w.ulo; j < w.uhi && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv) {
+            const int s = issued % STAGES;
+            const uint32_t ph = (issued / STAGES) & 1;
+            if (!bounded_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, p.wait_limit_ns)) {
+                ok = false;
+                break;
+            }
+            ptx::mbar_arrive_expect_tx(L::bar_kv_full(sbase, s), L::kTileBytes);
+#pragma unroll
+            for (int bx = 0; bx < kBoxes; ++bx)
+                ptx::tma_load_2d(sbase + L::kKV + s * L::kTileBytes + bx * L::kBoxBytes,
+                                 kv ? tm_v : tm_k, L::bar_kv_full(sbase, s), w.g * D + bx * 64,
+                                 w.start + j * kBN, pol_kv);
+            ++issued;
+        }
+    }
+    // Every copy issued must have landed before the block may exit.
+    drain_wait(L::bar_q(sbase), 0, p.wait_limit_ns);
+    const int first = issued > STAGES ? issued - STAGES : 0;
+    for (int i = first; i < issued; ++i)
+        drain_wait(L::bar_kv_full(sbase, i % STAGES), (i / STAGES) & 1, p.wait_limit_ns);
+}
+
+// ---------------------------------------------------------------- MMA issuer
+template <int D, int STAGES>
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, int slot) {
+    using L = SmemLayout<D, STAGES>;
+    constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, kBN, false, false);
+    const uint32_t qa = sbase + (x ? L::kQ1 : L::kQ0);
+    const uint32_t ka = sbase + L::kKV + slot * L::kTileBytes;
+    const uint32_t d_tmem = tmem + (x ? 128u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        // K-major, 128-byte swizzle: 16 elements (32 bytes) per step inside a
+        // 64-element box, the next box 16 KB further.
+        const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
+        ptx::mma_ss(d_tmem, ptx::smem_desc_sw128(qa + off, 16, 1024),
+                    ptx::smem_desc_sw128(ka + off, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot,
+                                         bool accumulate) {
+    using L = SmemLayout<D, STAGES>;
+    // B = V is [keys, d] with d contiguous: MN-major operand.  Swizzle atoms of
+    // 8 keys x 64 values are 1 KB apart along the keys (SBO) and the second
+    // 64-value half of d sits one 16 KB box further (LBO).
+    constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, D, false, true);
+    const uint32_t va = sbase + L::kKV + slot * L::kTileBytes;
+    const uint32_t p_tmem = tmem + (x ? 128u : 0u) + kPOffset;
+    const uint32_t d_tmem = tmem + kTmemO0 + (x ? 128u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < kBN / 16; ++kk) {
+        ptx::mma_ts(d_tmem, p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 2048, L::kBoxBytes, 1024),
+                    kIdesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, uint32_t tmem,
+                                         uint32_t sbase, volatile int* abort_flag) {
+    using L = SmemLayout<D, STAGES>;
+    const unsigned long long lim = p.wait_limit_ns;
+    bool ok = bounded_wait(L::bar_q(sbase), 0, abort_flag, lim);
+    ptx::tc_fence_after_sync();
+    int pc[2] = {0, 0};
+    bool first[2] = {true, true};
+    // Issue order per key block j:  S0(j), PV1(j-1), S1(j), PV0(j).  Each
+    // softmax group then has the two products of the other tile to hide its
+    // exponentials behind.  S_x(j) overwrites the P_x(j-1) columns only after
+    // PV_x(j-1) was issued; tcgen05 MMAs from one thread execute in order.
+    for (int j = w.ulo; ok && j < w.uhi; ++j) {
+        const int kidx = 2 * (j - w.ulo), vidx = kidx + 1;
+        const int ks = kidx % STAGES, vs = vidx % STAGES;
+        if (!(ok = bounded_wait(L::bar_kv_full(sbase, ks), (kidx / STAGES) & 1, abort_flag, lim)))
+            break;
+        ptx::tc_fence_after_sync();
+        if (tile_active_at(w, 0, j)) {
+            issue_qk<D, STAGES>(tmem, sbase, 0, ks);
+            ptx::tc_commit(L::bar_s_full(sbase, 0));
+        }
+        if (j > w.ulo) {
+            const int pvs = (vidx - 2) % STAGES;
+            if (tile_active_at(w, 1, j - 1)) {
+                if (!(ok = bounded_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim)))
+                    break;
+                ++pc[1];
+                ptx::tc_fence_after_sync();
+                issue_pv<D, STAGES>(tmem, sbase, 1, pvs, !first[1]);
+                first[1] = false;
+                if (j - 1 == w.hi[1] - 1) ptx::tc_commit(L::bar_o_done(sbase, 1));
+            }
+            ptx::tc_commit(L::bar_kv_empty(sbase, pvs));
+        }
+        if (tile_active_at(w, 1, j)) {
+            issue_qk<D, STAGES>(tmem, sbase, 1, ks);
+            ptx::tc_commit(L::bar_s_full(sbase, 1));
+        }
+        ptx::tc_commit(L::bar_kv_empty(sbase, ks));
+        if (!(ok = bounded_wait(L::bar_kv_full(sbase, vs), (vidx / STAGES) & 1, abort_flag, lim)))
+            break;
+        ptx::tc_fence_after_sync();
+        if (tile_active_at(w, 0, j)) {
+            if (!(ok = bounded_wait(L::bar_p_ready(sbase, 0), pc[0] & 1, abort_flag, lim))) break;
+            ++pc[0];
+            ptx::tc_fence_after_sync();
+            issue_pv<D, STAGES>(tmem, sbase, 0, vs, !first[0]);
+            first[0] = false;
+            if (j == w.hi[0] - 1) ptx::tc_commit(L::bar_o_done(sbase, 0));
+        }
+    }
+    if (ok && w.uhi > w.ulo) {
+        const int j = w.uhi - 1;
+        const int vs = (2 * (j - w.ulo) + 1) % STAGES;
+        if (tile_active_at(w, 1, j)) {
+            ok = bounded_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim);
+            if (ok) {
+                ptx::tc_fence_after_sync();
+                issue_pv<D, STAGES>(tmem, sbase, 1, vs, !first[1]);
+                ptx::tc_commit(L::bar_o_done(sbase, 1));
+            }
+        }
+        ptx::tc_commit(L::bar_kv_empty(sbase, vs));
+    }
+    // All MMAs must be complete before tensor memory is released.
+    ptx::tc_commit(L::bar_mma_final(sbase));
+    drain_wait(L::bar_mma_final(sbase), 0, lim);
+}
+
+// ---------------------------------------------------------------- softmax
+template <int D, int STAGES>
+__device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams& p, int x,
+                                             int warp_in_group, int lane, uint32_t tmem,
+                                             uint32_t sbase, volatile int* abort_flag) {
+    using L = SmemLayout<D, STAGES>;
+    // Per-tile scalars (avoid dynamic indexing of the pair's small arrays).
+    const bool active = x ? w.active[1] : w.active[0];
+    if (!active) return;
+    const int r0 = x ? w.r0[1] : w.r0[0];
+    const int blk_lo = x ? w.lo[1] : w.lo[0];
+    const int blk_hi = x ? w.hi[1] : w.hi[0];
+    const int h = x ? w.h[1] : w.h[0];
+    const unsigned long long lim = p.wait_limit_ns;
+    const int row = r0 + warp_in_group * 32 + lane;  // row within the sequence
+    const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + (x ? 128u : 0u);
+    const uint32_t t_p = t_s + kPOffset;
+    const uint32_t t_o = tmem + lane_off + kTmemO0 + (x ? 128u : 0u);
+    const float sl2 = p.scale_log2;
+
+    // Visible keys of this row: [key_lo, key_hi] (inclusive), inside the sequence.
+    const int key_lo = p.left >= 0 ? (row - p.left > 0 ? row - p.left : 0) : 0;
+    long long khi = p.right >= 0 ? (long long)row + p.right : (long long)w.len - 1;
+    if (khi > (long long)w.len - 1) khi = (long long)w.len - 1;
+    const int key_hi = (int)khi;
+    // A block needs no element mask when every (row, key) pair of the tile is visible.
+    const int tile_last_row = r0 + kBM - 1;
+
+    float m_ref = -INFINITY;  // reference maximum, log2 units (score * scale * log2 e)
+    float l_sum = 0.0f;       // running sum of the fp32 weights 2^(x - m_ref)  -> LSE
+    float l_bf = 0.0f;        // running sum of the same weights rounded to bf16 -> O
+    bool ok = true;
+
+    for (int j = blk_lo; j < blk_hi; ++j) {
+        ok = __all_sync(0xffffffffu,
+                        bounded_wait(L::bar_s_full(sbase, x), (j - blk_lo) & 1, abort_flag, lim));
+        if (!ok) break;
+        ptx::tc_fence_after_sync();
+        uint32_t s[128];
+        ptx::tmem_ld128_sync(t_s, s);
+
+        const int k0 = j * kBN;
+        const bool full_block =
+            (k0 + kBN <= w.len) && (p.left < 0 || (long long)k0 >= (long long)tile_last_row - p.left) &&
+            (p.right < 0 || (long long)k0 + kBN - 1 <= (long long)r0 + p.right);
+        if (!full_block) {
+            const int c_lo = key_lo - k0, c_hi = key_hi - k0;
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c < c_lo || c > c_hi) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+            mx0 = fmaxf(mx0, __uint_as_float(s[c + 0]));
+            mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+            mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
+            mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+        }
+        const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+
+        // Online softmax (Step 3): move the reference maximum only when the
+        // block's maximum exceeds it by more than the threshold.
+        float alpha = 1.0f;
+        bool rescale_o = false;
+        if (m_blk > m_ref + kRescaleThreshold) {
+            alpha = ptx::ex2_approx(m_ref - m_blk);
+            rescale_o = (m_ref != -INFINITY);
+            l_sum *= alpha;
+            l_bf *= alpha;
+            m_ref = m_blk;
+        }
+        // Step 4: the partial output takes the same correction.  The previous
+        // PV product of this tile is complete: it was issued before this S.
+        if (__any_sync(0xffffffffu, rescale_o)) {
+            const float a = rescale_o ? alpha : 1.0f;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                ptx::tmem_ld32_sync(t_o + cc * 32, o);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+                ptx::tmem_st32(t_o + cc * 32, o);
+            }
+        }
+
+        const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+        // The PV product multiplies the bf16-rounded weights, so O is divided by
+        // the sum of exactly those (a normalised convex combination of V); the
+        // LSE uses the sum of the unrounded fp32 weights.
+        float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+        float rb0 = 0.f, rb1 = 0.f, rb2 = 0.f, rb3 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const int c = q * 32 + 2 * i;
+                const float p0 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 0]), sl2, neg_m));
+                const float p1 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, neg_m));
+                const float p2 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, neg_m));
+                const float p3 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, neg_m));
+                sum0 += p0;
+                sum1 += p1;
+                sum2 += p2;
+                sum3 += p3;
+                pk[i] = ptx::pack_bf16x2(p0, p1);
+                pk[i + 1] = ptx::pack_bf16x2(p2, p3);
+                rb0 += __uint_as_float(pk[i] << 16);
+                rb1 += __uint_as_float(pk[i] & 0xffff0000u);
+                rb2 += __uint_as_float(pk[i + 1] << 16);
+                rb3 += __uint_as_float(pk[i + 1] & 0xffff0000u);
+            }
+            ptx::tmem_st16(t_p + q * 16, pk);
+        }
+        l_sum += (sum0 + sum1) + (sum2 + sum3);
+        l_bf += (rb0 + rb1) + (rb2 + rb3);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before_sync();
+        ptx::mbar_arrive(L::bar_p_ready(sbase, x));
+    }
+
+    if (!ok) return;
+    // Epilogue (Step 4 and 5): wait for the last PV product, divide once by the
+    // sum, round to bf16, and store O and the log-sum-exp.
+    ok = __all_sync(0xffffffffu, bounded_wait(L::bar_o_done(sbase, x), 0, abort_flag, lim));
+    if (!ok) return;
+    ptx::tc_fence_after_sync();
+    const bool store = row < w.len;
+    const float inv = l_bf > 0.0f ? 1.0f / l_bf : 0.0f;
+    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
+                    ((size_t)(w.start + (store ? row : 0)) * p.Hq + h) * (size_t)D * 2;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        ptx::tmem_ld32_sync(t_o + cc * 32, o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            pk[i] = ptx::pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        if (store) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                ptx::st_global_v4(orow + cc * 64 + v * 16, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                                  pk[4 * v + 3]);
+        }
+    }
+    if (store) {
+        const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
+        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + w.start + row
+                                        : ((size_t)w.b * p.Hq + h) * p.N + row;
+        p.lse[idx] = lse;
+    }
+}
+
+// ---------------------------------------------------------------- kernel
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using L = SmemLayout<D, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = ptx::smem_addr(smem);
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    const TilePair w = decode_pair(blockIdx.x, p);
+    if (!w.active[0] && !w.active[1]) return;  // uniform over the block
+
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    if (warp == kWarpProducer && lane == 0) {
+        ptx::mbar_init(L::bar_q(sbase), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(L::bar_kv_full(sbase, s), 1);
+            ptx::mbar_init(L::bar_kv_empty(sbase, s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            ptx::mbar_init(L::bar_s_full(sbase, x), 1);
+            ptx::mbar_init(L::bar_p_ready(sbase, x), 128);
+            ptx::mbar_init(L::bar_o_done(sbase, x), 1);
+        }
+        ptx::mbar_init(L::bar_mma_final(sbase), 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 8) {
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
+        softmax_role<D, STAGES>(w, p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
+    } else {
+        ptx::setmaxnreg_dec<kRegsOther>();
+        if (warp == kWarpProducer) {
+            if (lane == 0) producer_role<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, sbase, abort_flag);
+            __syncwarp();
+        } else if (warp == kWarpMma) {
+            if (lane == 0) mma_role<D, STAGES>(w, p, tmem, sbase, abort_flag);
+            __syncwarp();
+        }
+    }
+
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// A block that waits on a barrier nothing will signal: proves that bounded
+// waits give up, record the timeout and return without faulting the GPU.
+__global__ void selftest_bounded_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(ptx::smem_addr(&bar), 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    bounded_wait(ptx::smem_addr(&bar), 0, &abort_flag, limit_ns);
+    __syncthreads();
+}
+
+}  // namespace attn

@@ -1,0 +1,135 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact fused attention forward pass.
+ *
+ * Operation ("FlashAttention", ozercemkelahmet.com/tools/flashattention,
+ * sections "What it is" and "How it works", Steps 1-5):
+ *     O = softmax(scale * Q K^T + mask) V,   LSE = log of each row's softmax
+ *     normaliser (natural log, including the scale)
+ * computed tile by tile with an online softmax, so the score matrix never
+ * reaches device memory.  The result is exact up to rounding order: inputs are
+ * bf16, scores, softmax statistics and the O accumulator are fp32, the weights
+ * P are rounded to bf16 for the second product ("How it works", Step 8), and O
+ * is rounded once to bf16 (round to nearest even).
+ *
+ * Masks ("Flash Attention" skill page, skillmd.com, "Workflow 2",
+ * window_size=(left, right) with -1 for no limit; explainer page, Step 6):
+ *     key j is visible to query i of the same sequence iff
+ *         (window_left  < 0 || j >= i - window_left) &&
+ *         (window_right < 0 || j <= i + window_right)
+ *     and causal != 0 forces window_right = 0.  Bounds are inclusive.
+ * Grouped / multi-query attention (explainer page, "Variants you may meet"):
+ *     query head h reads key/value head h / (Hq / Hkv); Hkv == 1 is MQA.
+ * Packed variable-length batches ("Flash Attention 2 in HuggingFace",
+ * cloudcodetree.com, "Stack it with sequence packing"): cu_seqlens holds
+ * cumulative sequence boundaries and attention never crosses them.
+ *
+ * Threading and ownership: every buffer belongs to the caller.  The library
+ * keeps no per-call state and allocates no device memory; calls are
+ * asynchronous on the given stream and may be issued from several host
+ * threads.  The only global state is one device-side status word per device
+ * (see attn_device_status).
+ */
+#ifndef EXACT_ATTENTION_B200_ATTN_H
+#define EXACT_ATTENTION_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t / CUstream; NULL means the legacy default stream */
+
+enum attn_status {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,          /* a required pointer is NULL                        */
+    ATTN_ERR_SHAPE = -2,         /* B, Hq, Hkv <= 0, N < 0, Hq % Hkv != 0, sizes that
+                                    overflow 32-bit coordinates, max_seqlen < 0      */
+    ATTN_ERR_WINDOW = -3,        /* window_left or window_right < -1                  */
+    ATTN_ERR_UNSUPPORTED = -4,   /* d not in {64, 128}, or the device is not sm_100   */
+    ATTN_ERR_ALIGN = -5,         /* q, k, v, o not 16-byte aligned or lse not 4-byte  */
+    ATTN_ERR_CUDA = -6,          /* a CUDA runtime / driver call failed               */
+    ATTN_ERR_SCALE = -7,         /* scale is not a finite number > 0                  */
+    ATTN_ERR_WORKSPACE = -8,     /* attn_fwd_host: workspace missing or too small     */
+    ATTN_ERR_DEVICE_TIMEOUT = -9 /* reported by attn_device_status(): a kernel wait
+                                    ran past its time limit and the kernel gave up   */
+};
+
+/*
+ * attn_fwd -- fused exact attention forward on device buffers.
+ *
+ * Dense mode (cu_seqlens == NULL): B sequences of N tokens each.
+ *   q   [B, N, Hq,  d] bf16      k, v [B, N, Hkv, d] bf16
+ *   o   [B, N, Hq,  d] bf16      lse  [B, Hq, N] fp32
+ *   max_seqlen is ignored.
+ * Packed mode (cu_seqlens != NULL): B sequences packed back to back,
+ *   N = total number of tokens = cu_seqlens[B].
+ *   cu_seqlens: device int32[B + 1], cu_seqlens[0] = 0, non-decreasing.
+ *   q   [N, Hq,  d] bf16         k, v [N, Hkv, d] bf16
+ *   o   [N, Hq,  d] bf16         lse  [Hq, N] fp32
+ *   max_seqlen >= the longest sequence (used only to size the launch).  The
+ *   host never reads cu_seqlens; its contents are the caller's responsibility.
+ * All tensors are contiguous (row-major in the order shown).
+ *   d: head dimension, 64 or 128.
+ *   scale: finite, > 0 (pass 1/sqrt(d) for the usual scaling).
+ *   causal: nonzero -> key j visible only if j <= i (overrides window_right).
+ *   window_left / window_right: -1 (unlimited) or >= 0.
+ *   stream: CUDA stream the work is ordered on.
+ * Returns ATTN_OK after enqueueing the kernel (or when N == 0, with nothing
+ * enqueued), or a negative attn_status; on error nothing is enqueued.
+ * Device-side failures (a bounded wait that timed out) are reported through
+ * attn_device_status() once the stream has been synchronised.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int N, int d, float scale, int causal, int window_left, int window_right,
+             const int32_t* cu_seqlens, int max_seqlen, struct CUstream_st* stream);
+
+/*
+ * attn_fwd_host_workspace_bytes -- device workspace needed by attn_fwd_host
+ * for these sizes (q, k, v, o, lse and cu_seqlens copies, 256-byte aligned).
+ * packed: nonzero when cu_seqlens will be passed.  Returns 0 on bad sizes.
+ */
+size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int packed);
+
+/*
+ * attn_fwd_host -- the same operation on HOST buffers.
+ * Copies q, k, v (and cu_seqlens) host -> device into the caller's device
+ * workspace, runs attn_fwd on it, and copies o and lse device -> host, all
+ * ordered on `stream`.  The call returns after enqueueing; the host outputs
+ * are valid once the stream is synchronised.  Pinned (page-locked) host
+ * buffers make the copies asynchronous.  The layouts are those of attn_fwd;
+ * cu_seqlens is a host int32[B + 1] array here.
+ * workspace: device buffer of at least attn_fwd_host_workspace_bytes(...).
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                  int window_right, const int32_t* cu_seqlens, int max_seqlen, void* workspace,
+                  size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Static text for a status code (never NULL). */
+const char* attn_status_string(int status);
+
+/*
+ * attn_device_status -- read and clear the status word of the current device.
+ * Call after synchronising the streams that ran attn_fwd.  Returns ATTN_OK,
+ * ATTN_ERR_DEVICE_TIMEOUT if any kernel since the last call gave up on a
+ * bounded wait (its outputs are then undefined), or ATTN_ERR_CUDA if the word
+ * could not be read.
+ */
+int attn_device_status(void);
+
+/*
+ * attn_selftest_bounded_wait -- health check of the kernels' failure path.
+ * Launches one tiny block that waits on a barrier nothing will ever signal,
+ * with a limit of limit_ns nanoseconds (clamped to [1 us, 2 s]); the wait
+ * must give up, record ATTN_ERR_DEVICE_TIMEOUT in the status word and return.
+ * The GPU is never faulted or hung.  Returns the launch status.
+ */
+int attn_selftest_bounded_wait(uint64_t limit_ns, struct CUstream_st* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_B200_ATTN_H */

@@ -1,0 +1,251 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small cases are compared element by element against a full oracle run; the
+five named workloads are compared on sampled rows at full size, in the launch
+configuration the benchmark times.  The visible-key pattern is checked
+bit-exactly with a probe input (Q = 0 makes every visible weight equal, so
+exp(LSE) is the integer number of visible keys and O counts residues of the
+visible key indices)."""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_142_b200 as ea
+import workloads as W
+from gpu_helpers import (TOL_LSE, TOL_O, compare_full, default_scale, gpu_run, lse_index, o_index,
+                         oracle_run, sample_rows, visible_counts)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_attention_142_b200 import build
+    build.build()
+    ea.load_library()
+
+
+# (name, B, Hq, Hkv, N, d, causal, left, right, seed)
+DENSE_CASES = [
+    ("cfg1_noncausal_d64", 1, 2, 2, 256, 64, False, -1, -1, 0),
+    ("mha_causal_ragged", 2, 4, 4, 300, 128, True, -1, -1, 5),
+    ("gqa4_causal_ragged", 1, 8, 2, 520, 128, True, -1, -1, 6),
+    ("gqa3_rowpairs", 2, 6, 2, 333, 64, True, -1, -1, 7),
+    ("mqa_noncausal", 1, 4, 1, 257, 128, False, -1, -1, 8),
+    ("swa_causal", 1, 2, 2, 700, 128, True, 100, 0, 9),
+    ("window_both_sides", 1, 2, 2, 600, 64, False, 50, 70, 10),
+    ("window_right_only", 1, 4, 2, 400, 128, False, -1, 5, 11),
+    ("window_zero", 1, 2, 1, 300, 128, False, 0, 0, 12),
+    ("window_left_huge", 1, 2, 2, 260, 128, False, 1 << 30, 3, 13),
+    ("n1", 3, 2, 2, 1, 128, True, -1, -1, 14),
+    ("n127", 1, 2, 2, 127, 64, True, -1, -1, 15),
+    ("n128", 1, 4, 4, 128, 128, False, -1, -1, 16),
+    ("n129", 1, 4, 2, 129, 128, True, -1, -1, 17),
+    ("many_blocks", 1, 2, 2, 1100, 128, True, -1, -1, 18),
+    ("large_scores", 1, 2, 2, 384, 128, False, -1, -1, 19),
+]
+
+
+@pytest.mark.parametrize("case", DENSE_CASES, ids=lambda c: c[0])
+def test_dense_parity(case):
+    name, B, Hq, Hkv, N, d, causal, left, right, seed = case
+    q, k, v = W.draw_qkv((B, N, Hq, d), (B, N, Hkv, d), seed)
+    if name == "large_scores":
+        q = (q.float() * 4).to(torch.bfloat16)  # score spread of ~ +-50: exercises rescaling
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=causal,
+              window_left=left, window_right=right)
+    o, lse = gpu_run(q, k, v, **kw)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    compare_full(o, lse, o_ref, lse_ref)
+
+
+PACKED_CASES = [
+    # (name, lengths, Hq, Hkv, d, causal, left, right, seed)
+    ("packed_causal_gqa", [1, 0, 5, 128, 129, 300, 77], 4, 2, 128, True, -1, -1, 21),
+    ("packed_noncausal", [200, 3, 0, 0, 256, 131], 2, 2, 64, False, -1, -1, 22),
+    ("packed_window", [400, 129, 1, 600], 4, 1, 128, True, 64, 0, 23),
+    ("packed_single", [513], 2, 2, 128, True, -1, -1, 24),
+]
+
+
+@pytest.mark.parametrize("case", PACKED_CASES, ids=lambda c: c[0])
+def test_packed_parity(case):
+    name, lengths, Hq, Hkv, d, causal, left, right, seed = case
+    cu = W.cumulative(lengths)
+    T = cu[-1]
+    q, k, v = W.draw_qkv((T, Hq, d), (T, Hkv, d), seed)
+    kw = dict(B=len(lengths), Hq=Hq, Hkv=Hkv, N=T, d=d, scale=default_scale(d), causal=causal,
+              window_left=left, window_right=right, cu_seqlens=cu)
+    o, lse = gpu_run(q, k, v, **kw)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    compare_full(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_workload_sampled_rows(cfg):
+    """Full-size workloads in the benchmark's launch configuration; the oracle
+    computes sampled rows one by one."""
+    w = W.workload(cfg)
+    q, k, v = W.inputs(w)
+    kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d, scale=w.scale, causal=w.causal,
+              window_left=w.window_left, window_right=w.window_right, cu_seqlens=w.cu_seqlens)
+    o, lse = gpu_run(q, k, v, max_seqlen=w.max_seqlen, **kw)
+    lengths = ([b - a for a, b in zip(w.cu_seqlens[:-1], w.cu_seqlens[1:])] if w.packed
+               else [w.N] * w.B)
+    rows = sample_rows(lengths, w.Hq, n_random=600, seed=100 + cfg)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, rows=rows, **kw)
+    of = o.reshape(-1, w.Hq, w.d)
+    lf = lse.reshape(-1)
+    got_o = np.stack([of[o_index(w.cu_seqlens, b, i, w.N), h].to(torch.float64).numpy()
+                      for b, h, i in rows])
+    got_l = np.array([float(lf[lse_index(w.cu_seqlens, b, h, i, w.Hq, w.N)]) for b, h, i in rows])
+    dO = np.abs(got_o - o_ref).max()
+    dL = np.abs(got_l - lse_ref).max()
+    assert dO <= TOL_O, dO
+    assert dL <= TOL_LSE, dL
+    # every row was written, and nothing is NaN/inf
+    assert torch.isfinite(o.float()).all()
+    assert torch.isfinite(lse).all()
+
+
+def _mask_probe(lengths, Hq, Hkv, d, causal, left, right, packed):
+    """Q = 0 and V[t, c] = [t mod d == c]: every visible weight is equal, so
+    exp(LSE) is the number of visible keys and O[i, c] is the fraction of
+    visible keys whose index is c modulo d."""
+    B = len(lengths)
+    if packed:
+        cu = W.cumulative(lengths)
+        T = cu[-1]
+        shape_q, shape_kv = (T, Hq, d), (T, Hkv, d)
+        N = T
+    else:
+        cu = None
+        N = lengths[0]
+        T = B * N
+        shape_q, shape_kv = (B, N, Hq, d), (B, N, Hkv, d)
+    g = torch.Generator().manual_seed(77)
+    q = torch.zeros(shape_q, dtype=torch.bfloat16)
+    k = torch.randn(shape_kv, generator=g).to(torch.bfloat16)
+    t = torch.arange(T).reshape(-1, 1) % d
+    onehot = (t == torch.arange(d).reshape(1, -1)).to(torch.bfloat16)  # [T, d]
+    v = onehot.reshape(T, 1, d).expand(T, Hkv, d).reshape(shape_kv).contiguous()
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=causal,
+              window_left=left, window_right=right, cu_seqlens=cu)
+    o, lse = gpu_run(q, k, v, **kw)
+    # 1) exact visible-key counts for every row, from exp(LSE)
+    counts = visible_counts(lengths, causal, left, right)
+    lse_np = lse.to(torch.float64).numpy()
+    for b, L in enumerate(lengths):
+        for h in range(Hq):
+            if L == 0:
+                continue
+            if packed:
+                row_lse = lse_np[h, cu[b]:cu[b] + L]
+            else:
+                row_lse = lse_np[b, h, :L]
+            got = np.rint(np.exp(row_lse)).astype(np.int64)
+            bad = np.nonzero(got != counts[b])[0]
+            assert bad.size == 0, f"seq {b} head {h}: rows {bad[:8]} count {got[bad[:8]]} != {counts[b][bad[:8]]}"
+    # 2) which keys: O equals the oracle's residue fractions on sampled rows
+    rows = sample_rows(lengths, Hq, n_random=300, seed=5)
+    o_ref, _, nvis = oracle_run(q, k, v, rows=rows, **kw)
+    of = o.reshape(-1, Hq, d)
+    for r, (b, h, i) in enumerate(rows):
+        got = of[o_index(cu, b, i, N), h].to(torch.float64).numpy()
+        # exact value count/n rounded once to bf16; allow one bf16 ulp
+        ref = o_ref[r]
+        ulp = np.where(ref > 0, 2.0 ** (np.floor(np.log2(np.maximum(ref, 1e-30))) - 7), 0.0)
+        assert np.all(np.abs(got - ref) <= ulp + 1e-12), (b, h, i)
+
+
+@pytest.mark.parametrize("probe", [
+    ("causal_dense", [1000, 1000], 2, 2, 128, True, -1, -1, False),
+    ("window_dense", [1500], 4, 2, 128, True, 300, 0, False),
+    ("window_two_sided_d64", [900], 2, 1, 64, False, 129, 40, False),
+    ("noncausal_dense", [700, 700], 2, 2, 64, False, -1, -1, False),
+    ("packed_causal", [5, 0, 130, 1, 513, 255], 4, 2, 128, True, -1, -1, True),
+    ("packed_window", [600, 129, 2], 2, 2, 128, True, 127, 0, True),
+], ids=lambda p: p[0])
+def test_mask_pattern_bit_exact(probe):
+    _, lengths, Hq, Hkv, d, causal, left, right, packed = probe
+    _mask_probe(lengths, Hq, Hkv, d, causal, left, right, packed)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_mask_pattern_workloads(cfg):
+    """The same probe at the named workloads' full shapes and masks."""
+    w = W.workload(cfg)
+    lengths = ([b - a for a, b in zip(w.cu_seqlens[:-1], w.cu_seqlens[1:])] if w.packed
+               else [w.N] * w.B)
+    Hq = min(w.Hq, 8)
+    Hkv = max(1, Hq * w.Hkv // w.Hq)
+    _mask_probe(lengths, Hq, Hkv, w.d, w.causal, w.window_left, w.window_right, w.packed)
+
+
+def test_causal_row0_is_v0_exactly():
+    B, N, H, d = 2, 300, 4, 128
+    q, k, v = W.draw_qkv((B, N, H, d), (B, N, H, d), 31)
+    o, _ = gpu_run(q, k, v, B=B, Hq=H, Hkv=H, N=N, d=d, scale=default_scale(d), causal=True)
+    assert torch.equal(o[:, 0], v[:, 0])
+
+
+def test_deterministic():
+    B, N, Hq, Hkv, d = 1, 777, 8, 2, 128
+    q, k, v = W.draw_qkv((B, N, Hq, d), (B, N, Hkv, d), 32)
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=True)
+    o1, l1 = gpu_run(q, k, v, **kw)
+    o2, l2 = gpu_run(q, k, v, **kw)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_host_entry_matches_device_entry():
+    lengths = [300, 1, 129]
+    cu = W.cumulative(lengths)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 128
+    q, k, v = W.draw_qkv((T, Hq, d), (T, Hkv, d), 33)
+    kw = dict(B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=default_scale(d), causal=True,
+              window_left=-1, window_right=-1, cu_seqlens=cu)
+    o_dev, l_dev = gpu_run(q, k, v, **kw)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((Hq, T), dtype=torch.float32).pin_memory()
+    cuh = torch.tensor(cu, dtype=torch.int32)
+    nbytes = ea.attn_fwd_host_workspace_bytes(3, Hq, Hkv, T, d, True)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ea.attn_fwd_host(qh, kh, vh, oh, lh, 3, Hq, Hkv, T, d, default_scale(d), True, -1, -1, cuh,
+                     0, ws, nbytes)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o_dev) and torch.equal(lh, l_dev)
+
+
+def test_bounded_wait_reports_timeout_and_recovers():
+    assert ea.attn_device_status() == ea.ATTN_OK
+    assert ea.attn_selftest_bounded_wait(2_000_000) == ea.ATTN_OK  # 2 ms limit
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_ERR_DEVICE_TIMEOUT
+    assert ea.attn_device_status() == ea.ATTN_OK  # read clears it
+    # the context is healthy: a normal call still matches the oracle
+    B, N, H, d = 1, 200, 2, 64
+    q, k, v = W.draw_qkv((B, N, H, d), (B, N, H, d), 34)
+    kw = dict(B=B, Hq=H, Hkv=H, N=N, d=d, scale=default_scale(d), causal=True)
+    o, lse = gpu_run(q, k, v, **kw)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    compare_full(o, lse, o_ref, lse_ref)
+
+
+def test_empty_inputs_enqueue_nothing():
+    z = torch.empty(0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(0, dtype=torch.float32, device="cuda")
+    assert ea.attn_fwd(z, z, z, z, lse, 2, 4, 2, 0, 128, 0.1, True) == ea.ATTN_OK
+    cu = torch.zeros(4, dtype=torch.int32, device="cuda")
+    assert ea.attn_fwd(z, z, z, z, lse, 3, 4, 2, 0, 128, 0.1, True, cu_seqlens=cu,
+                       max_seqlen=0) == ea.ATTN_OK
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+
+
+def test_wrong_device_arch_is_not_silently_used():
+    major, minor = torch.cuda.get_device_capability()
+    assert (major, minor) == (10, 0), "these kernels are built for sm_100a only"
