@@ -8,6 +8,7 @@
 //   warp  8    producer: TMA loads of Q (once) and of the K/V ring
 //   warp  9    MMA issuer: tcgen05 S = Q K^T (both operands in shared memory)
 //              and O += P V (P read from tensor memory)
+//   (both run converged over all 32 lanes; one elected lane issues)
 //   warps 10-11 spare (complete the third warpgroup)
 // Registers move from the third warpgroup to the two softmax warpgroups with
 // setmaxnreg (the whole score row of a query lives in one thread).
@@ -37,6 +38,7 @@
 #include <cuda.h>
 
 #include "attn.h"
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 
 namespace attn {
@@ -60,7 +62,35 @@ constexpr float kLn2 = 0.693147180559945309f;
 constexpr uint32_t kRegsSoftmax = 216;
 constexpr uint32_t kRegsOther = 72;
 
+// One in kPolyPeriod groups of four weights takes its exponential from the
+// FMA-pipe polynomial instead of the MUFU unit (whose rate equals the tensor
+// core's at d = 128 and would otherwise be the bottleneck).
+constexpr int kPolyPeriod = 8;
+
 enum : int { kPairHeads = 0, kPairRows = 1 };
+
+// 2^x for a pair of arguments x <= 8 on the FMA/ALU pipes:
+// n = rint(x) via the 1.5 * 2^23 rounding constant, f = x - n in [-1/2, 1/2]
+// (exact), 2^f by the fitted cubic, and n added to the exponent bits.
+// Arguments below -125 are clamped (their weight becomes ~2^-125, far below
+// the fp32 resolution of any row sum, which is >= 1).
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const uint64_t x = ptx::f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = ptx::fadd2(x, ptx::f2_pack(kRound, kRound));
+    const uint64_t n = ptx::fadd2(t, ptx::f2_pack(-kRound, -kRound));
+    const uint64_t f = ptx::ffma2(n, ptx::f2_pack(-1.0f, -1.0f), x);
+    uint64_t p = ptx::ffma2(f, ptx::f2_pack(exp2poly::kC3, exp2poly::kC3),
+                            ptx::f2_pack(exp2poly::kC2, exp2poly::kC2));
+    p = ptx::ffma2(p, f, ptx::f2_pack(exp2poly::kC1, exp2poly::kC1));
+    p = ptx::ffma2(p, f, ptx::f2_pack(1.0f, 1.0f));
+    float p0, p1, t0, t1;
+    ptx::f2_unpack(p, p0, p1);
+    ptx::f2_unpack(t, t0, t1);
+    // the low bits of t hold n; shifted by 23 they are n in the exponent field
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
 
 struct FwdParams {
     void* o;
@@ -146,6 +176,12 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity,
     return true;
 }
 
+// bounded_wait by every lane of a warp, with a warp-uniform outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns) {
+    return __all_sync(0xffffffffu, bounded_wait(bar, parity, abort_flag, limit_ns));
+}
+
 // The two query tiles of one CTA and the key blocks each of them needs.
 struct TilePair {
     int b, start, len, g;
@@ -225,11 +261,11 @@ __device__ __forceinline__ void producer_role(const TilePair& w, const FwdParams
     const uint64_t pol_q = ptx::policy_evict_first();
     const uint64_t pol_kv = ptx::policy_evict_last();
 
-    ptx::mbar_arrive_expect_tx(L::bar_q(sbase), 2 * L::kTileBytes);
+    ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * L::kTileBytes);
     for (int x = 0; x < 2; ++x) {
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx)
-            ptx::tma_load_2d(sbase + (x ? L::kQ1 : L::kQ0) + bx * L::kBoxBytes, tm_q,
+            ptx::tma_load_2d_elect(sbase + (x ? L::kQ1 : L::kQ0) + bx * L::kBoxBytes, tm_q,
                              L::bar_q(sbase), w.h[x] * D + bx * 64, w.start + w.r0[x], pol_q);
     }
 
@@ -239,14 +275,14 @@ __device__ __forceinline__ void producer_role(const TilePair& w, const FwdParams
         for (int kv = 0; kv < 2; ++kv) {
             const int s = issued % STAGES;
             const uint32_t ph = (issued / STAGES) & 1;
-            if (!bounded_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, p.wait_limit_ns)) {
+            if (!warp_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, p.wait_limit_ns)) {
                 ok = false;
                 break;
             }
-            ptx::mbar_arrive_expect_tx(L::bar_kv_full(sbase, s), L::kTileBytes);
+            ptx::mbar_arrive_expect_tx_elect(L::bar_kv_full(sbase, s), L::kTileBytes);
 #pragma unroll
             for (int bx = 0; bx < kBoxes; ++bx)
-                ptx::tma_load_2d(sbase + L::kKV + s * L::kTileBytes + bx * L::kBoxBytes,
+                ptx::tma_load_2d_elect(sbase + L::kKV + s * L::kTileBytes + bx * L::kBoxBytes,
                                  kv ? tm_v : tm_k, L::bar_kv_full(sbase, s), w.g * D + bx * 64,
                                  w.start + j * kBN, pol_kv);
             ++issued;
@@ -272,7 +308,7 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, i
         // K-major, 128-byte swizzle: 16 elements (32 bytes) per step inside a
         // 64-element box, the next box 16 KB further.
         const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
-        ptx::mma_ss(d_tmem, ptx::smem_desc_sw128(qa + off, 16, 1024),
+        ptx::mma_ss_elect(d_tmem, ptx::smem_desc_sw128(qa + off, 16, 1024),
                     ptx::smem_desc_sw128(ka + off, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
     }
 }
@@ -290,7 +326,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
     const uint32_t d_tmem = tmem + kTmemO0 + (x ? 128u : 0u);
 #pragma unroll
     for (int kk = 0; kk < kBN / 16; ++kk) {
-        ptx::mma_ts(d_tmem, p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 2048, L::kBoxBytes, 1024),
+        ptx::mma_ts_elect(d_tmem, p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 2048, L::kBoxBytes, 1024),
                     kIdesc, (accumulate || kk > 0) ? 1u : 0u);
     }
 }
@@ -300,7 +336,7 @@ __device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, 
                                          uint32_t sbase, volatile int* abort_flag) {
     using L = SmemLayout<D, STAGES>;
     const unsigned long long lim = p.wait_limit_ns;
-    bool ok = bounded_wait(L::bar_q(sbase), 0, abort_flag, lim);
+    bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
     ptx::tc_fence_after_sync();
     int pc[2] = {0, 0};
     bool first[2] = {true, true};
@@ -311,58 +347,58 @@ __device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, 
     for (int j = w.ulo; ok && j < w.uhi; ++j) {
         const int kidx = 2 * (j - w.ulo), vidx = kidx + 1;
         const int ks = kidx % STAGES, vs = vidx % STAGES;
-        if (!(ok = bounded_wait(L::bar_kv_full(sbase, ks), (kidx / STAGES) & 1, abort_flag, lim)))
+        if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (kidx / STAGES) & 1, abort_flag, lim)))
             break;
         ptx::tc_fence_after_sync();
         if (tile_active_at(w, 0, j)) {
             issue_qk<D, STAGES>(tmem, sbase, 0, ks);
-            ptx::tc_commit(L::bar_s_full(sbase, 0));
+            ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
         }
         if (j > w.ulo) {
             const int pvs = (vidx - 2) % STAGES;
             if (tile_active_at(w, 1, j - 1)) {
-                if (!(ok = bounded_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim)))
+                if (!(ok = warp_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim)))
                     break;
                 ++pc[1];
                 ptx::tc_fence_after_sync();
                 issue_pv<D, STAGES>(tmem, sbase, 1, pvs, !first[1]);
                 first[1] = false;
-                if (j - 1 == w.hi[1] - 1) ptx::tc_commit(L::bar_o_done(sbase, 1));
+                if (j - 1 == w.hi[1] - 1) ptx::tc_commit_elect(L::bar_o_done(sbase, 1));
             }
-            ptx::tc_commit(L::bar_kv_empty(sbase, pvs));
+            ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
         }
         if (tile_active_at(w, 1, j)) {
             issue_qk<D, STAGES>(tmem, sbase, 1, ks);
-            ptx::tc_commit(L::bar_s_full(sbase, 1));
+            ptx::tc_commit_elect(L::bar_s_full(sbase, 1));
         }
-        ptx::tc_commit(L::bar_kv_empty(sbase, ks));
-        if (!(ok = bounded_wait(L::bar_kv_full(sbase, vs), (vidx / STAGES) & 1, abort_flag, lim)))
+        ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
+        if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), (vidx / STAGES) & 1, abort_flag, lim)))
             break;
         ptx::tc_fence_after_sync();
         if (tile_active_at(w, 0, j)) {
-            if (!(ok = bounded_wait(L::bar_p_ready(sbase, 0), pc[0] & 1, abort_flag, lim))) break;
+            if (!(ok = warp_wait(L::bar_p_ready(sbase, 0), pc[0] & 1, abort_flag, lim))) break;
             ++pc[0];
             ptx::tc_fence_after_sync();
             issue_pv<D, STAGES>(tmem, sbase, 0, vs, !first[0]);
             first[0] = false;
-            if (j == w.hi[0] - 1) ptx::tc_commit(L::bar_o_done(sbase, 0));
+            if (j == w.hi[0] - 1) ptx::tc_commit_elect(L::bar_o_done(sbase, 0));
         }
     }
     if (ok && w.uhi > w.ulo) {
         const int j = w.uhi - 1;
         const int vs = (2 * (j - w.ulo) + 1) % STAGES;
         if (tile_active_at(w, 1, j)) {
-            ok = bounded_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim);
+            ok = warp_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim);
             if (ok) {
                 ptx::tc_fence_after_sync();
                 issue_pv<D, STAGES>(tmem, sbase, 1, vs, !first[1]);
-                ptx::tc_commit(L::bar_o_done(sbase, 1));
+                ptx::tc_commit_elect(L::bar_o_done(sbase, 1));
             }
         }
-        ptx::tc_commit(L::bar_kv_empty(sbase, vs));
+        ptx::tc_commit_elect(L::bar_kv_empty(sbase, vs));
     }
     // All MMAs must be complete before tensor memory is released.
-    ptx::tc_commit(L::bar_mma_final(sbase));
+    ptx::tc_commit_elect(L::bar_mma_final(sbase));
     drain_wait(L::bar_mma_final(sbase), 0, lim);
 }
 
@@ -420,11 +456,11 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
         }
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-            mx0 = fmaxf(mx0, __uint_as_float(s[c + 0]));
-            mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
-            mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
-            mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+        for (int c = 0; c < 128; c += 8) {
+            mx0 = ptx::fmax3(mx0, __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
+            mx1 = ptx::fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+            mx2 = ptx::fmax3(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+            mx3 = ptx::fmax3(mx3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
         }
         const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
 
@@ -454,36 +490,55 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
         }
 
         const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+        const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+        const uint64_t negm_2 = ptx::f2_pack(neg_m, neg_m);
         // The PV product multiplies the bf16-rounded weights, so O is divided by
         // the sum of exactly those (a normalised convex combination of V); the
         // LSE uses the sum of the unrounded fp32 weights.
-        float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
-        float rb0 = 0.f, rb1 = 0.f, rb2 = 0.f, rb3 = 0.f;
+        uint64_t sum_a = 0, sum_b = 0;  // fp32 weights, packed pairs
+        float rb0 = 0.f, rb1 = 0.f, rb2 = 0.f, rb3 = 0.f;  // bf16-rounded weights
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
                 const int c = q * 32 + 2 * i;
-                const float p0 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 0]), sl2, neg_m));
-                const float p1 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, neg_m));
-                const float p2 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, neg_m));
-                const float p3 = ptx::ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, neg_m));
-                sum0 += p0;
-                sum1 += p1;
-                sum2 += p2;
-                sum3 += p3;
+                float x0, x1, x2, x3;
+                ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(__uint_as_float(s[c + 0]), __uint_as_float(s[c + 1])),
+                                          sl2_2, negm_2), x0, x1);
+                ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])),
+                                          sl2_2, negm_2), x2, x3);
+                float p0, p1, p2, p3;
+                if ((i / 2) % kPolyPeriod == kPolyPeriod - 1) {
+                    exp2_poly_pair(x0, x1, p0, p1);
+                    exp2_poly_pair(x2, x3, p2, p3);
+                } else {
+                    p0 = ptx::ex2_approx(x0);
+                    p1 = ptx::ex2_approx(x1);
+                    p2 = ptx::ex2_approx(x2);
+                    p3 = ptx::ex2_approx(x3);
+                }
+                sum_a = ptx::fadd2(sum_a, ptx::f2_pack(p0, p1));
+                sum_b = ptx::fadd2(sum_b, ptx::f2_pack(p2, p3));
                 pk[i] = ptx::pack_bf16x2(p0, p1);
                 pk[i + 1] = ptx::pack_bf16x2(p2, p3);
-                rb0 += __uint_as_float(pk[i] << 16);
-                rb1 += __uint_as_float(pk[i] & 0xffff0000u);
-                rb2 += __uint_as_float(pk[i + 1] << 16);
-                rb3 += __uint_as_float(pk[i + 1] & 0xffff0000u);
+                if ((i / 2) % 2 == 0) {
+                    rb0 = ptx::add_bf16x2_to_f32(rb0, pk[i]);
+                    rb1 = ptx::add_bf16x2_to_f32(rb1, pk[i + 1]);
+                } else {
+                    rb2 = ptx::add_bf16x2_to_f32(rb2, pk[i]);
+                    rb3 = ptx::add_bf16x2_to_f32(rb3, pk[i + 1]);
+                }
             }
             ptx::tmem_st16(t_p + q * 16, pk);
         }
-        l_sum += (sum0 + sum1) + (sum2 + sum3);
-        l_bf += (rb0 + rb1) + (rb2 + rb3);
+        {
+            float a0, a1, b0, b1;
+            ptx::f2_unpack(sum_a, a0, a1);
+            ptx::f2_unpack(sum_b, b0, b1);
+            l_sum += (a0 + a1) + (b0 + b1);
+            l_bf += (rb0 + rb1) + (rb2 + rb3);
+        }
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_p_ready(sbase, x));
@@ -574,11 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (warp == kWarpProducer) {
-            if (lane == 0) producer_role<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, sbase, abort_flag);
-            __syncwarp();
+            producer_role<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, sbase, abort_flag);
         } else if (warp == kWarpMma) {
-            if (lane == 0) mma_role<D, STAGES>(w, p, tmem, sbase, abort_flag);
-            __syncwarp();
+            mma_role<D, STAGES>(w, p, tmem, sbase, abort_flag);
         }
     }
 
