@@ -237,6 +237,29 @@ __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]
         : "memory");
 }
 
+// 64 consecutive columns per thread, then wait.
+__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&r)[64]) {
+#define ATTN_R32B(b)                                                                        \
+    "=r"(r[b + 0]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]),           \
+        "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7]), "=r"(r[b + 8]), "=r"(r[b + 9]),      \
+        "=r"(r[b + 10]), "=r"(r[b + 11]), "=r"(r[b + 12]), "=r"(r[b + 13]), "=r"(r[b + 14]), \
+        "=r"(r[b + 15]), "=r"(r[b + 16]), "=r"(r[b + 17]), "=r"(r[b + 18]), "=r"(r[b + 19]), \
+        "=r"(r[b + 20]), "=r"(r[b + 21]), "=r"(r[b + 22]), "=r"(r[b + 23]), "=r"(r[b + 24]), \
+        "=r"(r[b + 25]), "=r"(r[b + 26]), "=r"(r[b + 27]), "=r"(r[b + 28]), "=r"(r[b + 29]), \
+        "=r"(r[b + 30]), "=r"(r[b + 31])
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : ATTN_R32B(0), ATTN_R32B(32)
+        : "r"(taddr)
+        : "memory");
+#undef ATTN_R32B
+}
+
 // Four 32-column loads (128 columns) with a single wait at the end.
 __device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
 #define ATTN_R32(b)                                                                         \
@@ -263,6 +286,14 @@ __device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[12
         : "r"(taddr)
         : "memory");
 #undef ATTN_R32
+}
+
+// 32 lanes x 32 bits, 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
 }
 
 // 32 lanes x 32 bits, 16 consecutive columns per thread.
