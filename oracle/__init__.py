@@ -54,6 +54,15 @@ def load(path: Optional[str] = None):
         ctypes.c_int, ctypes.c_int, ctypes.c_int,  # causal left right
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,  # cu rows nrows threads
     ]
+    lib.oracle_attn_kvcache.restype = ctypes.c_int
+    lib.oracle_attn_kvcache.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # q kc vc
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # o lse nvis
+        ctypes.c_void_p, ctypes.c_void_p,  # cache_seqlens block_table
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,  # B Hq Hkv Nq d
+        ctypes.c_int, ctypes.c_int, ctypes.c_double,  # page_size pages_per_seq scale
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,  # causal left right threads
+    ]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -114,4 +123,31 @@ def attn_fwd(q, k, v, *, B: int, Hq: int, Hkv: int, N: int, d: int, scale: float
         None if cu is None else cu.ctypes.data, rows_p, nrows, int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd failed with code {rc}")
+    return o, lse, nvis
+
+
+def attn_kvcache(q, k_cache, v_cache, cache_seqlens, *, B: int, Hq: int, Hkv: int, Nq: int,
+                 d: int, page_size: int, pages_per_seq: int, scale: float,
+                 causal: bool = True, window_left: int = -1, window_right: int = -1,
+                 block_table=None, nthreads: int = 0, lib=None):
+    """Newest-token attention against a (paged) key/value cache.
+
+    q [B, Nq, Hq, d] bf16 bits; caches [num_pages, page_size, Hkv, d] bf16 bits;
+    cache_seqlens int32 [B]; block_table int32 [B, pages_per_seq] or None
+    (contiguous cache).  Returns o [B, Nq, Hq, d] fp64, lse [B, Hq, Nq], nvis.
+    """
+    lib = lib or load()
+    q, k_cache, v_cache = _bits(q), _bits(k_cache), _bits(v_cache)
+    cs = np.ascontiguousarray(np.asarray(cache_seqlens, dtype=np.int32))
+    bt = None if block_table is None else np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    o = np.empty((B, Nq, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq, Nq), dtype=np.float64)
+    nvis = np.empty((B, Hq, Nq), dtype=np.int64)
+    rc = lib.oracle_attn_kvcache(q.ctypes.data, k_cache.ctypes.data, v_cache.ctypes.data,
+                                 o.ctypes.data, lse.ctypes.data, nvis.ctypes.data, cs.ctypes.data,
+                                 None if bt is None else bt.ctypes.data, B, Hq, Hkv, Nq, d,
+                                 page_size, pages_per_seq, float(scale), int(bool(causal)),
+                                 int(window_left), int(window_right), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_kvcache failed with code {rc}")
     return o, lse, nvis

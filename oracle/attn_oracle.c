@@ -226,3 +226,113 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/*
+ * oracle_attn_kvcache -- attention of the newest tokens against a key/value
+ * cache ("FlashAttention" explainer page, How it works, Step 9: decoding with a
+ * cache of past keys and values, one or a few new tokens at a time).
+ *
+ * Sequence b holds L_b = cache_seqlens[b] keys (the new tokens included); its
+ * Nq query rows are the newest positions pos_i = L_b - Nq + i (so causal
+ * masking is aligned to the end of the cache).  Key j is visible to query i iff
+ *     (left < 0 || j >= pos_i - left) && (right < 0 || j <= pos_i + right),
+ * causal forcing right = 0, j < L_b.
+ *   q        [B, Nq, Hq, d]  bf16 bits
+ *   k/v cache, pages of page_size rows: [num_pages, page_size, Hkv, d] bf16;
+ *            logical key j of sequence b lives in page block_table[b * pages_per_seq
+ *            + j / page_size] at row j % page_size; block_table == NULL means page
+ *            b * pages_per_seq + j / page_size (a contiguous [B, pages_per_seq *
+ *            page_size, Hkv, d] cache).
+ *   o        [B, Nq, Hq, d] fp64,   lse [B, Hq, Nq] fp64,   nvis like lse (or NULL)
+ * Requires L_b >= Nq for every sequence.
+ */
+int oracle_attn_kvcache(const uint16_t *q, const uint16_t *kc, const uint16_t *vc,
+                        double *o, double *lse, int64_t *nvis,
+                        const int32_t *cache_seqlens, const int32_t *block_table,
+                        int B, int Hq, int Hkv, int Nq, int d, int page_size,
+                        int pages_per_seq, double scale, int causal, int window_left,
+                        int window_right, int nthreads) {
+    if (!q || !kc || !vc || !o || !lse || !cache_seqlens) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || d <= 0 || page_size <= 0 ||
+        pages_per_seq <= 0)
+        return ORACLE_ERR_ARG;
+    if (Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    const int group = Hq / Hkv;
+    const int64_t left = window_left;
+    const int64_t right = causal ? 0 : window_right;
+    int64_t maxL = 0;
+    for (int b = 0; b < B; ++b) {
+        const int64_t L = cache_seqlens[b];
+        if (L < Nq || L > (int64_t)page_size * pages_per_seq) return ORACLE_ERR_ARG;
+        if (L > maxL) maxL = L;
+    }
+#ifdef _OPENMP
+    const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#else
+    (void)nthreads;
+#endif
+    int failed = 0;
+#pragma omp parallel num_threads(nt)
+    {
+        double *s_row = (double *)malloc(sizeof(double) * (size_t)(maxL > 0 ? maxL : 1));
+        if (!s_row) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int b = 0; b < B; ++b) {
+            for (int h = 0; h < Hq; ++h) {
+                if (!s_row) continue;
+                const int g = h / group;
+                const int64_t L = cache_seqlens[b];
+                for (int i = 0; i < Nq; ++i) {
+                    const int64_t pos = L - Nq + i;
+                    const uint16_t *qi = q + (((int64_t)b * Nq + i) * Hq + h) * d;
+                    double *o_row = o + (((int64_t)b * Nq + i) * Hq + h) * d;
+                    double M = -INFINITY;
+                    int64_t n = 0;
+                    for (int64_t j = 0; j < L; ++j) {
+                        if (!key_visible(pos, j, left, right)) {
+                            s_row[j] = -INFINITY;
+                            continue;
+                        }
+                        const int64_t page = block_table
+                                                 ? block_table[(int64_t)b * pages_per_seq + j / page_size]
+                                                 : (int64_t)b * pages_per_seq + j / page_size;
+                        const int64_t row = page * page_size + j % page_size;
+                        const uint16_t *kj = kc + (row * Hkv + g) * d;
+                        double dot = 0.0;
+                        for (int t = 0; t < d; ++t) dot += widen_bf16(qi[t]) * widen_bf16(kj[t]);
+                        s_row[j] = scale * dot;
+                        if (s_row[j] > M) M = s_row[j];
+                        ++n;
+                    }
+                    const int64_t li = ((int64_t)b * Hq + h) * Nq + i;
+                    if (nvis) nvis[li] = n;
+                    if (n == 0) {
+                        for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+                        lse[li] = -INFINITY;
+                        continue;
+                    }
+                    double Z = 0.0;
+                    for (int64_t j = 0; j < L; ++j)
+                        if (s_row[j] != -INFINITY) Z += exp(s_row[j] - M);
+                    for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+                    for (int64_t j = 0; j < L; ++j) {
+                        if (s_row[j] == -INFINITY) continue;
+                        const double p = exp(s_row[j] - M) / Z;
+                        const int64_t page = block_table
+                                                 ? block_table[(int64_t)b * pages_per_seq + j / page_size]
+                                                 : (int64_t)b * pages_per_seq + j / page_size;
+                        const int64_t row = page * page_size + j % page_size;
+                        const uint16_t *vj = vc + (row * Hkv + g) * d;
+                        for (int c = 0; c < d; ++c) o_row[c] += p * widen_bf16(vj[c]);
+                    }
+                    lse[li] = M + log(Z);
+                }
+            }
+        }
+        free(s_row);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

@@ -383,6 +383,126 @@ def pin_rows_mode_matches_full(lib):
         assert lse2[r] == lse[h, t] and nv2[r] == nv[h, t]
 
 
+# --------------------------------------------------------------------------
+# key/value cache (decode) entry
+# --------------------------------------------------------------------------
+def _kvcache_inputs(rng, B, Hq, Hkv, Nq, d, lens, page_size, pages_per_seq, paged):
+    """Random caches laid out in pages; returns q, kc, vc, block_table."""
+    num_pages = B * pages_per_seq
+    q = _bf16(rng.standard_normal((B, Nq, Hq, d)))
+    kc = _bf16(rng.standard_normal((num_pages, page_size, Hkv, d)))
+    vc = _bf16(rng.standard_normal((num_pages, page_size, Hkv, d)))
+    bt = None
+    if paged:
+        bt = rng.permutation(num_pages).astype(np.int32).reshape(B, pages_per_seq)
+    return q, kc, vc, bt
+
+
+def _gather_cache(c, bt, b, L, page_size, pages_per_seq):
+    """Logical [L, H, d] rows of sequence b from a paged cache (torch tensor)."""
+    rows = []
+    for j in range(L):
+        page = bt[b, j // page_size] if bt is not None else b * pages_per_seq + j // page_size
+        rows.append(c[int(page), j % page_size])
+    return torch.stack(rows)
+
+
+def pin_kvcache_matches_forward_last_rows(lib):
+    """Decoding the newest tokens equals the last rows of full causal attention."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, d, page_size, pps = 2, 4, 2, 16, 8, 5
+    lens = [37, 19]
+    for Nq in (1, 3):
+        q, kc, vc, _ = _kvcache_inputs(rng, B, Hq, Hkv, Nq, d, lens, page_size, pps, False)
+        o, lse, _ = oracle.attn_kvcache(W.bf16_bits(q), W.bf16_bits(kc), W.bf16_bits(vc), lens,
+                                        B=B, Hq=Hq, Hkv=Hkv, Nq=Nq, d=d, page_size=page_size,
+                                        pages_per_seq=pps, scale=0.4, causal=True, lib=lib)
+        for b, L in enumerate(lens):
+            kf = _gather_cache(kc, None, b, L, page_size, pps).unsqueeze(0).contiguous()
+            vf = _gather_cache(vc, None, b, L, page_size, pps).unsqueeze(0).contiguous()
+            qf = torch.zeros((1, L, Hq, d), dtype=torch.bfloat16)
+            qf[0, L - Nq:] = q[b]
+            of, lf, _ = _run(lib, qf, kf, vf, B=1, Hq=Hq, Hkv=Hkv, N=L, d=d, scale=0.4, causal=True)
+            assert np.array_equal(o[b], of.reshape(L, Hq, d)[L - Nq:])
+            assert np.array_equal(lse[b], lf[0][:, L - Nq:])
+
+
+def pin_kvcache_paged_equals_contiguous(lib):
+    rng = np.random.default_rng(32)
+    B, Hq, Hkv, Nq, d, page_size, pps = 3, 4, 4, 2, 8, 4, 6
+    lens = [24, 2, 13]
+    q, kc, vc, bt = _kvcache_inputs(rng, B, Hq, Hkv, Nq, d, lens, page_size, pps, True)
+    # contiguous copy of the same logical cache
+    kcont = torch.zeros_like(kc)
+    vcont = torch.zeros_like(vc)
+    for b in range(B):
+        for p_ in range(pps):
+            kcont[b * pps + p_] = kc[int(bt[b, p_])]
+            vcont[b * pps + p_] = vc[int(bt[b, p_])]
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, Nq=Nq, d=d, page_size=page_size, pages_per_seq=pps, scale=0.5,
+              causal=True, window_left=7, lib=lib)
+    o1, l1, _ = oracle.attn_kvcache(W.bf16_bits(q), W.bf16_bits(kc), W.bf16_bits(vc), lens,
+                                    block_table=bt, **kw)
+    o2, l2, _ = oracle.attn_kvcache(W.bf16_bits(q), W.bf16_bits(kcont), W.bf16_bits(vcont), lens,
+                                    **kw)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def pin_kvcache_uniform_closed_form(lib):
+    """Q = 0: O is the mean of V over the visible keys, aligned to the end of
+    the cache; LSE = ln(count)."""
+    rng = np.random.default_rng(33)
+    B, Hq, Hkv, Nq, d, page_size, pps = 2, 2, 1, 3, 4, 4, 4
+    lens = [11, 16]
+    for causal, left, right in [(True, -1, -1), (True, 3, 0), (False, 2, 1), (False, -1, -1)]:
+        q = torch.zeros((B, Nq, Hq, d), dtype=torch.bfloat16)
+        kc = _bf16(rng.standard_normal((B * pps, page_size, Hkv, d)))
+        vc = _bf16(rng.integers(-6, 7, size=(B * pps, page_size, Hkv, d)))
+        o, lse, nv = oracle.attn_kvcache(W.bf16_bits(q), W.bf16_bits(kc), W.bf16_bits(vc), lens,
+                                         B=B, Hq=Hq, Hkv=Hkv, Nq=Nq, d=d, page_size=page_size,
+                                         pages_per_seq=pps, scale=1.0, causal=causal,
+                                         window_left=left, window_right=right, lib=lib)
+        for b, L in enumerate(lens):
+            vf = _gather_cache(vc, None, b, L, page_size, pps)[:, 0].to(torch.float64).numpy()
+            for i in range(Nq):
+                pos = L - Nq + i
+                lo = 0 if left < 0 else max(0, pos - left)
+                r_ = 0 if causal else right
+                hi = L - 1 if r_ < 0 else min(L - 1, pos + r_)
+                for h in range(Hq):
+                    assert nv[b, h, i] == hi - lo + 1
+                    assert np.allclose(o[b, i, h], vf[lo:hi + 1].mean(axis=0), rtol=0, atol=1e-13)
+                    assert abs(lse[b, h, i] - math.log(hi - lo + 1)) <= 1e-13
+
+
+def pin_kvcache_torch_sdpa(lib):
+    import torch.nn.functional as F
+    rng = np.random.default_rng(34)
+    B, Hq, Hkv, Nq, d, page_size, pps = 2, 6, 2, 4, 32, 16, 4
+    lens = [50, 37]
+    q, kc, vc, bt = _kvcache_inputs(rng, B, Hq, Hkv, Nq, d, lens, page_size, pps, True)
+    scale = d ** -0.5
+    o, lse, _ = oracle.attn_kvcache(W.bf16_bits(q), W.bf16_bits(kc), W.bf16_bits(vc), lens,
+                                    B=B, Hq=Hq, Hkv=Hkv, Nq=Nq, d=d, page_size=page_size,
+                                    pages_per_seq=pps, scale=scale, causal=True, window_left=20,
+                                    block_table=bt, lib=lib)
+    for b, L in enumerate(lens):
+        kf = _gather_cache(kc, bt, b, L, page_size, pps).to(torch.float64)  # [L, Hkv, d]
+        vf = _gather_cache(vc, bt, b, L, page_size, pps).to(torch.float64)
+        g = Hq // Hkv
+        kt = torch.repeat_interleave(kf, g, dim=1).transpose(0, 1)  # [Hq, L, d]
+        vt = torch.repeat_interleave(vf, g, dim=1).transpose(0, 1)
+        qt = q[b].to(torch.float64).transpose(0, 1)  # [Hq, Nq, d]
+        # end-aligned causal band with a left window of 20, built from tril/triu
+        full = _band_mask(L, True, 20, 0)  # [L, L] for queries at every position
+        mask = full[L - Nq:]  # the newest Nq query positions
+        ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+        assert np.abs(o[b] - ref.transpose(0, 1).numpy()).max() <= 1e-12
+        sc = (qt @ kt.transpose(-1, -2)) * scale
+        ref_lse = torch.logsumexp(sc.masked_fill(~mask, float("-inf")), dim=-1).numpy()
+        assert np.abs(lse[b] - ref_lse).max() <= 1e-12
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_uniform_scores,
@@ -397,4 +517,8 @@ ALL_PINS = [
     pin_gqa_equals_repeated,
     pin_torch_sdpa,
     pin_rows_mode_matches_full,
+    pin_kvcache_matches_forward_last_rows,
+    pin_kvcache_paged_equals_contiguous,
+    pin_kvcache_uniform_closed_form,
+    pin_kvcache_torch_sdpa,
 ]

@@ -29,6 +29,11 @@ MUTANTS = {
     "packed_lse_layout": ("(int64_t)h * tokens + start + i", "(int64_t)h * tokens + i"),
     "k_row_transposed": ("const uint16_t *kj = k + ((start + j) * (int64_t)Hkv + g) * d;",
                          "const uint16_t *kj = k + ((start + (i + j) % L) * (int64_t)Hkv + g) * d;"),
+    "kvcache_top_left_alignment": ("const int64_t pos = L - Nq + i;", "const int64_t pos = i;"),
+    "kvcache_block_table_ignored": ("                        const int64_t page = block_table\n                                                 ? block_table[(int64_t)b * pages_per_seq + j / page_size]",
+                                    "                        const int64_t page = 0\n                                                 ? block_table[(int64_t)b * pages_per_seq + j / page_size]"),
+    "kvcache_page_row_swapped": ("const int64_t row = page * page_size + j % page_size;\n                        const uint16_t *vj",
+                                 "const int64_t row = page * page_size + (page_size - 1 - j % page_size);\n                        const uint16_t *vj"),
 }
 
 
