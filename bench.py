@@ -1,7 +1,8 @@
 #!/usr/bin/env python3
 """Benchmark of the fused attention forward (one JSON line on stdout).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5|decode]
+                    [--impl reference]
 
 A step is one call of the fused forward (the whole hot path) over one batch of
 the workload.  The default workload is the causal grouped-query forward at
@@ -22,6 +23,13 @@ collective on the data path.
 
 --impl reference times the CPU oracle (fp64, all host cores) on bounded
 samples of the same workload (rank 0 only).
+
+--workload decode times the key/value-cache decode instead (attn_decode: one
+new token for each of 64 sequences against 8192-token paged caches, 32 query
+heads over 8 key/value heads, d = 128).  It is bound by HBM, so its metric is
+GB/s of algorithmic bytes (every visible cached key and value read once, plus
+q, o and lse) against the measured copy bandwidth; a step is one attn_decode
+call (the slice kernel and, with more than one slice, the merge kernel).
 """
 from __future__ import annotations
 
@@ -49,6 +57,9 @@ METRIC = "attn fwd TFLOP/s (bf16, causal, d=128) and % of B200 dense BF16 peak"
 UNIT = "TFLOP/s"
 SPEC_BF16_TFLOPS = 2250.0   # NVIDIA datasheet dense bf16, for context
 FALLBACK_BF16_TFLOPS = 1590.0
+DECODE_METRIC = "attn decode GB/s (bf16 paged KV cache, d=128) and % of measured HBM bandwidth"
+DECODE_UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["exact_attention_142_b200/csrc/attn_fwd_kernel.cuh",
                   "exact_attention_142_b200/csrc/ptx.cuh",
                   "exact_attention_142_b200/csrc/attn_api.cu"]
@@ -275,6 +286,235 @@ def run_cuda(args, w: W.Workload, rank: int, world: int, local_rank: int):
 
 
 # ---------------------------------------------------------------------------
+# key/value-cache decode
+# ---------------------------------------------------------------------------
+def decode_visible_keys(w: W.DecodeWorkload) -> int:
+    """Cached keys that at least one query row of a sequence sees, summed over
+    sequences (each is read once per key/value head)."""
+    right = 0 if w.causal else w.window_right
+    total = 0
+    for L in w.lengths:
+        lo = 0 if w.window_left < 0 else max(0, L - w.Nq - w.window_left)
+        hi = L - 1 if right < 0 else min(L - 1, L - 1 + right)
+        total += max(0, hi - lo + 1)
+    return total
+
+
+def decode_bytes(w: W.DecodeWorkload) -> float:
+    kv = 2.0 * decode_visible_keys(w) * w.Hkv * w.d * 2
+    qo = 2.0 * w.B * w.Nq * w.Hq * w.d * 2
+    return kv + qo + 4.0 * w.B * w.Hq * w.Nq
+
+
+def run_decode(args, w: W.DecodeWorkload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_142_b200 as ea
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    q, kc, vc, seqlens, table = W.decode_inputs(w, device="cuda")
+    sd, td = seqlens.to(dev), table.to(dev) if table is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    splits = args.splits or ea.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Nq, w.max_len)
+    nbytes = ea.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.d, w.page_size,
+                                            w.pages_per_seq, splits)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_decode(q, kc, vc, o, lse, sd, td, w.B, w.Hq, w.Hkv, w.Nq, w.d, w.page_size,
+                       w.pages_per_seq, w.scale, w.causal, w.window_left, w.window_right, splits,
+                       ws if nbytes else None, nbytes, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.mark_end()
+    kernel_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported a failure during the timed region")
+
+    # end to end: pinned host inputs copied in, result copied out, every step
+    host = [t.cpu().pin_memory() for t in (q, kc, vc, seqlens)]
+    host_table = table.pin_memory() if table is not None else None
+    oh = torch.empty(tuple(o.shape), dtype=o.dtype).pin_memory()
+    lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+    devs = [q, kc, vc, sd]
+
+    def e2e_step():
+        for hsrc, ddst in zip(host, devs):
+            ddst.copy_(hsrc, non_blocking=True)
+        if host_table is not None:
+            td.copy_(host_table, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(3, min(args.steps, 10))
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(e_steps):
+        es[i].record(stream)
+        e2e_step()
+        ee[i].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es, ee)) / e_steps
+    h2d = sum(t.numel() * t.element_size() for t in host) + (
+        host_table.numel() * 4 if host_table is not None else 0)
+    d2h = oh.numel() * 2 + lh.numel() * 4
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([kernel_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        kernel_ms, e2e_ms = float(t[0]), float(t[1])
+    launches = args.steps * (2 if nbytes else 1)
+    return kernel_ms, e2e_ms, h2d, d2h, clocks, splits, launches
+
+
+def decode_oracle_sample(w: W.DecodeWorkload, inputs, nseq: int, seed: int):
+    """Time the oracle on `nseq` sequences drawn from the workload; returns
+    (seconds, algorithmic bytes of those sequences, threads)."""
+    import oracle
+    q, kc, vc, seqlens, table = inputs
+    rng = np.random.default_rng(seed)
+    pick = np.sort(rng.choice(w.B, size=nseq, replace=False))
+    sub = W.DecodeWorkload("sample", nseq, w.Hq, w.Hkv, w.Nq, w.d, w.page_size, w.pages_per_seq,
+                           [w.lengths[b] for b in pick], w.paged, w.causal, w.window_left,
+                           w.window_right, w.seed)
+    t0 = time.perf_counter()
+    oracle.attn_kvcache(W.bf16_bits(q[pick]), W.bf16_bits(kc), W.bf16_bits(vc),
+                        seqlens.numpy()[pick], B=nseq, Hq=w.Hq, Hkv=w.Hkv, Nq=w.Nq, d=w.d,
+                        page_size=w.page_size, pages_per_seq=w.pages_per_seq, scale=w.scale,
+                        causal=w.causal, window_left=w.window_left, window_right=w.window_right,
+                        block_table=None if table is None else table.numpy()[pick])
+    return time.perf_counter() - t0, decode_bytes(sub), oracle.num_threads()
+
+
+def decode_host_inputs(w: W.DecodeWorkload):
+    """The benchmark's inputs (drawn with the CUDA generator) brought to the host."""
+    return tuple(t.cpu() if t is not None else None for t in W.decode_inputs(w, device="cuda"))
+
+
+def decode_cpu_baseline(w: W.DecodeWorkload, inputs, target_s: float = 12.0):
+    dt, by, thr = decode_oracle_sample(w, inputs, 1, seed=1)
+    nseq = int(max(1, min(w.B, round(target_s / max(dt, 1e-6)))))
+    dt, by, thr = decode_oracle_sample(w, inputs, nseq, seed=2)
+    return {"value": by / dt / 1e9, "unit": DECODE_UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{nseq} of {w.B} sequences (all heads, full caches), fp64 oracle, "
+                      f"{dt:.1f} s on {thr} threads"}
+
+
+def decode_config(w: W.DecodeWorkload, n_gpus: int, splits: int):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "d": w.d,
+            "cache_len": max(w.lengths), "page_size": w.page_size, "paged": w.paged,
+            "causal": w.causal, "window": [w.window_left, w.window_right],
+            "num_splits": splits, "bytes_per_step": decode_bytes(w),
+            "l2": "flushed between timed steps (the caches are 17x L2 as well)",
+            "parallelism": f"replicas x{n_gpus} (no collective)"}
+
+
+def main_decode(args, rank, world, local_rank):
+    w = W.decode_workload()
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inputs = decode_host_inputs(w)
+        budget_s = 150.0 / max(1, args.steps + args.warmup)
+        dt, _, _ = decode_oracle_sample(w, inputs, 1, seed=1)
+        nseq = int(max(1, min(w.B, round(min(budget_s, 30.0) / max(dt, 1e-6)))))
+        for i in range(args.warmup):
+            decode_oracle_sample(w, inputs, nseq, seed=10 + i)
+        tot_t, tot_b, thr = 0.0, 0.0, 1
+        for i in range(args.steps):
+            dt, by, thr = decode_oracle_sample(w, inputs, nseq, seed=1000 + i)
+            tot_t += dt
+            tot_b += by
+        value = tot_b / tot_t / 1e9
+        print(json.dumps({
+            "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": decode_config(w, args.gpus, 0), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": DECODE_UNIT, "cores": thr, "kind": "oracle",
+                             "sample": f"{nseq} sequences per step; fp64 oracle on {thr} threads"},
+            "e2e": {"value": value, "unit": DECODE_UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        kernel_ms, e2e_ms, h2d, d2h, clocks, splits, launches = run_decode(
+            args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.barrier()
+    if rank == 0:
+        by = decode_bytes(w)
+        achieved = by / (kernel_ms * 1e-3) / 1e9
+        peaks, src = measured_peaks()
+        peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        line = {
+            "metric": DECODE_METRIC, "value": achieved * world, "unit": DECODE_UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": kernel_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal bf16 q and caches, random page table)",
+            "config": decode_config(w, world, splits),
+            "e2e": {"value": by * world / (e2e_ms * 1e-3) / 1e9, "unit": DECODE_UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{src} hbm_gbs (copy)" if src == "measured"
+                         else "fallback 6650 GB/s",
+                         "kernel": "attn_decode_split<128,4>"
+                                   + (" + attn_decode_combine<128>" if splits > 1 else ""),
+                         "timed_as": "whole attn_decode call (both kernels)"},
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = decode_cpu_baseline(w, decode_host_inputs(w))
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
 # oracle (CPU) timing
 # ---------------------------------------------------------------------------
 def oracle_sample(w: W.Workload, q, k, v, nrows: int, seed: int):
@@ -356,17 +596,22 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--workload", default="3", choices=["1", "2", "3", "4", "5", "decode"])
+    ap.add_argument("--splits", type=int, default=0,
+                    help="decode only: cache slices (0 = attn_decode_default_splits)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = W.workload(args.workload)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload == "decode":
+        main_decode(args, rank, world, local_rank)
+        return
+    w = W.workload(int(args.workload))
 
     if args.impl == "reference":
         if rank == 0:

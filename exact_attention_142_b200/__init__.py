@@ -8,7 +8,8 @@ outputs with torch and calls ``attn_fwd``.
 from ._binding import (  # noqa: F401
     ATTN_ERR_ALIGN, ATTN_ERR_CUDA, ATTN_ERR_DEVICE_TIMEOUT, ATTN_ERR_NULL, ATTN_ERR_SCALE,
     ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WINDOW, ATTN_ERR_WORKSPACE, ATTN_OK, AttnError,
-    attn_device_status, attn_fwd, attn_fwd_host, attn_fwd_host_workspace_bytes,
+    attn_decode, attn_decode_default_splits, attn_decode_workspace_bytes, attn_device_status,
+    attn_fwd, attn_fwd_host, attn_fwd_host_workspace_bytes,
     attn_selftest_bounded_wait, attn_status_string, library_path, load_library)
 
 
@@ -37,4 +38,34 @@ def attention(q, k, v, *, causal=False, window_left=-1, window_right=-1, scale=N
         scale = 1.0 / math.sqrt(d)
     attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window_left, window_right,
              cu_seqlens, max_seqlen, stream)
+    return o, lse
+
+
+def attention_with_kvcache(q, k_cache, v_cache, cache_seqlens, *, block_table=None, causal=True,
+                           window_left=-1, window_right=-1, scale=None, num_splits=0,
+                           stream=None):
+    """Newest-token attention against a (paged) key/value cache via attn_decode.
+
+    q [B, Nq, Hq, d]; caches [num_pages, page_size, Hkv, d]; cache_seqlens int32
+    [B] and block_table int32 [B, pages_per_seq] (or None: contiguous cache, then
+    num_pages = B * pages_per_seq) on the device.  num_splits <= 0 picks
+    attn_decode_default_splits.  Returns o [B, Nq, Hq, d], lse [B, Hq, Nq].
+    """
+    import math
+
+    import torch
+    B, Nq, Hq, d = q.shape
+    page_size, Hkv = k_cache.shape[1], k_cache.shape[2]
+    pages_per_seq = block_table.shape[1] if block_table is not None else k_cache.shape[0] // B
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits <= 0:
+        num_splits = attn_decode_default_splits(B, Hq, Hkv, Nq, page_size * pages_per_seq)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, page_size, pages_per_seq, num_splits)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq, d,
+                page_size, pages_per_seq, scale, causal, window_left, window_right, num_splits,
+                ws, nbytes, stream)
     return o, lse

@@ -44,8 +44,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         newest = max(os.path.getmtime(s) for s in srcs)
         if os.path.getmtime(LIB) >= newest:
             return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp",
-           os.path.join(CSRC, "attn_api.cu")]
+    units = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp", *units]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)

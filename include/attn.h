@@ -107,6 +107,45 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
                   int window_right, const int32_t* cu_seqlens, int max_seqlen, void* workspace,
                   size_t workspace_bytes, struct CUstream_st* stream);
 
+/*
+ * attn_decode -- attention of the newest tokens against a key/value cache,
+ * split along the cache ("FlashAttention" explainer page, How it works, Step 9:
+ * decoding with a cache of past keys and values; the split partials are merged
+ * by the online-softmax rule of "Long context beyond a single GPU").
+ *
+ *   q       [B, Nq, Hq, d] bf16: the Nq (1..16) newest tokens of each sequence
+ *   k_cache, v_cache [num_pages, page_size, Hkv, d] bf16 (paged cache)
+ *   block_table  device int32 [B, pages_per_seq]: page of logical page p of
+ *           sequence b; NULL means page b * pages_per_seq + p, i.e. a contiguous
+ *           cache [B, pages_per_seq * page_size, Hkv, d].
+ *   cache_seqlens device int32 [B]: keys held by sequence b, the new tokens
+ *           included (Nq <= cache_seqlens[b] <= page_size * pages_per_seq).
+ *   o       [B, Nq, Hq, d] bf16;  lse [B, Hq, Nq] fp32 (natural log).
+ * Query row i of sequence b sits at position pos = cache_seqlens[b] - Nq + i;
+ * key j is visible iff (window_left < 0 || j >= pos - window_left) &&
+ * (window_right < 0 || j <= pos + window_right), causal forcing window_right = 0.
+ *   num_splits: number of slices of the cache (>= 1; see
+ *           attn_decode_default_splits).  With more than one slice, partial
+ *           results go to `workspace` (device, 256-byte aligned, at least
+ *           attn_decode_workspace_bytes(...) bytes; may be NULL when that is 0).
+ * Asynchronous on `stream`; allocates nothing.  The host never reads
+ * cache_seqlens or block_table; their contents are the caller's responsibility.
+ * Returns ATTN_OK or a negative attn_status (ATTN_ERR_UNSUPPORTED for Nq > 16).
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                const int32_t* cache_seqlens, const int32_t* block_table, int B, int Hq, int Hkv,
+                int Nq, int d, int page_size, int pages_per_seq, float scale, int causal,
+                int window_left, int window_right, int num_splits, void* workspace,
+                size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Device workspace attn_decode needs for these sizes (0 when one slice). */
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int page_size,
+                                   int pages_per_seq, int num_splits);
+
+/* A slice count that gives about four CTAs per SM, with at least 256 keys per
+ * slice (max_cache_len = page_size * pages_per_seq). */
+int attn_decode_default_splits(int B, int Hq, int Hkv, int Nq, int max_cache_len);
+
 /* Static text for a status code (never NULL). */
 const char* attn_status_string(int status);
 

@@ -106,3 +106,60 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_binding, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         _binding.load_library()
+
+
+def call_decode(**over):
+    args = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, o=FAKE, lse=FAKE, cache_seqlens=FAKE,
+                block_table=None, B=2, Hq=8, Hkv=2, Nq=1, d=128, page_size=16, pages_per_seq=8,
+                scale=0.1, causal=1, window_left=-1, window_right=-1, num_splits=1,
+                workspace=None, workspace_bytes=0, stream=0)
+    args.update(over)
+    return ea.attn_decode(check=False, **args)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=0), ea.ATTN_ERR_SHAPE),
+    (dict(Nq=0), ea.ATTN_ERR_SHAPE),
+    (dict(Hq=6, Hkv=4), ea.ATTN_ERR_SHAPE),
+    (dict(page_size=0), ea.ATTN_ERR_SHAPE),
+    (dict(pages_per_seq=0), ea.ATTN_ERR_SHAPE),
+    (dict(num_splits=0), ea.ATTN_ERR_SHAPE),
+    (dict(page_size=1 << 20, pages_per_seq=1 << 12), ea.ATTN_ERR_SHAPE),  # > 2^31 keys
+    (dict(window_left=-3), ea.ATTN_ERR_WINDOW),
+    (dict(d=80), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(Nq=17), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), ea.ATTN_ERR_SCALE),
+    (dict(cache_seqlens=None), ea.ATTN_ERR_NULL),
+    (dict(v_cache=None), ea.ATTN_ERR_NULL),
+    (dict(k_cache=FAKE + 4), ea.ATTN_ERR_ALIGN),
+    (dict(lse=FAKE + 1), ea.ATTN_ERR_ALIGN),
+    (dict(num_splits=4), ea.ATTN_ERR_WORKSPACE),          # 128 keys -> 2 slices, no workspace
+    (dict(num_splits=4, workspace=FAKE, workspace_bytes=16), ea.ATTN_ERR_WORKSPACE),
+    (dict(num_splits=4, workspace=FAKE + 16, workspace_bytes=1 << 20), ea.ATTN_ERR_WORKSPACE),
+])
+def test_decode_validation_codes(lib, over, code):
+    assert call_decode(**over) == code
+
+
+def test_decode_workspace_size(lib):
+    r = lambda x: (x + 255) // 256 * 256
+    B, Hq, Hkv, Nq, d = 3, 16, 4, 2, 128
+    # 1000 keys in 4 slices -> 256 keys per slice (a multiple of the 64-key tile) -> 4 slices
+    got = ea.attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, 100, 10, 4)
+    rows = B * Nq * Hq
+    assert got == r(4 * rows * d * 4) + r(4 * rows * 4)
+    # 7 slices of 1000 keys -> ceil(143 / 64) * 64 = 192 keys -> 6 slices
+    assert ea.attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, 100, 10, 7) == \
+        r(6 * rows * d * 4) + r(6 * rows * 4)
+    assert ea.attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, 100, 10, 1) == 0
+    assert ea.attn_decode_workspace_bytes(0, Hq, Hkv, Nq, d, 100, 10, 4) == 0
+
+
+def test_decode_default_splits(lib):
+    # few sequences and a long cache: many slices, at least 256 keys each
+    s = ea.attn_decode_default_splits(1, 32, 8, 1, 8192)
+    assert 8 <= s <= 32
+    assert ea.attn_decode_default_splits(1, 32, 8, 1, 300) == 1
+    # enough sequences to fill the GPU: one or two slices
+    assert ea.attn_decode_default_splits(256, 32, 8, 1, 8192) == 1
+    assert ea.attn_decode_default_splits(0, 32, 8, 1, 8192) == 1

@@ -126,3 +126,75 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
 def from_bits(a: np.ndarray) -> torch.Tensor:
     """Inverse of bf16_bits."""
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------
+# key/value-cache decode
+# --------------------------------------------------------------------------
+@dataclass
+class DecodeWorkload:
+    """Nq newest tokens per sequence against a paged key/value cache.
+
+    Caches are [B * pages_per_seq, page_size, Hkv, d]; the page table, when
+    `paged`, is a seeded random permutation of all pages (so logical neighbours
+    sit far apart in memory, as in a serving pool); otherwise sequence b owns
+    pages b * pages_per_seq ... contiguously.
+    """
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    d: int
+    page_size: int
+    pages_per_seq: int
+    lengths: List[int]
+    paged: bool
+    causal: bool
+    window_left: int
+    window_right: int
+    seed: int
+    scale: float = field(default=0.0)
+
+    def __post_init__(self):
+        if self.scale == 0.0:
+            self.scale = default_scale(self.d)
+
+    @property
+    def max_len(self) -> int:
+        return self.page_size * self.pages_per_seq
+
+
+def decode_workload() -> DecodeWorkload:
+    """The decode benchmark: 64 sequences, each with a full 8192-token cache,
+    one new token, the grouped-query head layout of the 8192-token causal
+    workload (32 query heads over 8 key/value heads, d = 128), 64-token pages."""
+    return DecodeWorkload("decode_gqa_b64_hq32_hkv8_l8192_d128_page64", 64, 32, 8, 1, 128, 64, 128,
+                          [8192] * 64, True, True, -1, -1, 5)
+
+
+def decode_inputs(w: DecodeWorkload, device: str = "cpu"):
+    """(q [B,Nq,Hq,d], k_cache, v_cache, cache_seqlens int32 [B],
+    block_table int32 [B, pages_per_seq] or None).  The draws follow the same
+    rule as draw_qkv (fp32 normal, rounded to bf16; q, k, v in that order),
+    then the page permutation; `device="cuda"` draws with a CUDA generator
+    (faster for multi-GB caches; different bytes than the CPU draw)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    pages = w.B * w.pages_per_seq
+    q = torch.randn((w.B, w.Nq, w.Hq, w.d), dtype=torch.float32, generator=g,
+                    device=device).to(torch.bfloat16)
+    kc = torch.empty((pages, w.page_size, w.Hkv, w.d), dtype=torch.bfloat16, device=device)
+    vc = torch.empty_like(kc)
+    for c in (kc, vc):  # page by page to bound the fp32 temporary
+        step = max(1, (1 << 26) // (w.page_size * w.Hkv * w.d))
+        for p0 in range(0, pages, step):
+            p1 = min(pages, p0 + step)
+            c[p0:p1] = torch.randn((p1 - p0, w.page_size, w.Hkv, w.d), dtype=torch.float32,
+                                   generator=g, device=device).to(torch.bfloat16)
+    seqlens = torch.tensor(w.lengths, dtype=torch.int32)
+    table = None
+    if w.paged:
+        perm = torch.randperm(pages, generator=torch.Generator().manual_seed(w.seed))
+        table = perm.to(torch.int32).reshape(w.B, w.pages_per_seq)
+    return q, kc, vc, seqlens, table
