@@ -63,6 +63,9 @@ FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["exact_attention_142_b200/csrc/attn_fwd_kernel.cuh",
                   "exact_attention_142_b200/csrc/ptx.cuh",
                   "exact_attention_142_b200/csrc/attn_api.cu"]
+DECODE_SOURCES = ["exact_attention_142_b200/csrc/attn_decode_kernel.cuh",
+                  "exact_attention_142_b200/csrc/ptx.cuh",
+                  "exact_attention_142_b200/csrc/attn_decode_api.cu"]
 
 
 def visible_pairs(w: W.Workload) -> int:
@@ -93,25 +96,25 @@ def measured_peaks():
         return {}, "fallback"
 
 
-def kernel_sources_digest() -> str:
+def kernel_sources_digest(sources=None) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name: str):
+def recorded_traffic(workload_name: str, prefix: str = "attn_fwd", sources=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload_name}_traffic.md")
+    path = os.path.join(ROOT, "profiles", f"{prefix}_{workload_name}_traffic.md")
     try:
         text = open(path).read()
     except OSError:
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     s = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_sources_digest():
+    if not m or not s or s.group(1) != kernel_sources_digest(sources):
         return None
     return float(m.group(1))
 
@@ -328,8 +331,8 @@ def run_decode(args, w: W.DecodeWorkload, rank: int, world: int, local_rank: int
 
     def step():
         ea.attn_decode(q, kc, vc, o, lse, sd, td, w.B, w.Hq, w.Hkv, w.Nq, w.d, w.page_size,
-                       w.pages_per_seq, w.scale, w.causal, w.window_left, w.window_right, splits,
-                       ws if nbytes else None, nbytes, stream)
+                       w.pages_per_seq, kc.shape[0], w.scale, w.causal, w.window_left,
+                       w.window_right, splits, ws if nbytes else None, nbytes, stream)
 
     for _ in range(args.warmup):
         step()
@@ -426,12 +429,17 @@ def decode_host_inputs(w: W.DecodeWorkload):
 
 
 def decode_cpu_baseline(w: W.DecodeWorkload, inputs, target_s: float = 12.0):
-    dt, by, thr = decode_oracle_sample(w, inputs, 1, seed=1)
-    nseq = int(max(1, min(w.B, round(target_s / max(dt, 1e-6)))))
-    dt, by, thr = decode_oracle_sample(w, inputs, nseq, seed=2)
-    return {"value": by / dt / 1e9, "unit": DECODE_UNIT, "cores": thr, "kind": "oracle",
-            "sample": f"{nseq} of {w.B} sequences (all heads, full caches), fp64 oracle, "
-                      f"{dt:.1f} s on {thr} threads"}
+    """The oracle on whole batches of the workload, repeated until about
+    target_s seconds of CPU work."""
+    tot_t, tot_b, reps, thr = 0.0, 0.0, 0, 1
+    while tot_t < target_s and reps < 1000:
+        dt, by, thr = decode_oracle_sample(w, inputs, w.B, seed=2 + reps)
+        tot_t += dt
+        tot_b += by
+        reps += 1
+    return {"value": tot_b / tot_t / 1e9, "unit": DECODE_UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{reps} passes over all {w.B} sequences (all heads, full caches), "
+                      f"fp64 oracle, {tot_t:.1f} s on {thr} threads"}
 
 
 def decode_config(w: W.DecodeWorkload, n_gpus: int, splits: int):
@@ -444,7 +452,7 @@ def decode_config(w: W.DecodeWorkload, n_gpus: int, splits: int):
 
 
 def main_decode(args, rank, world, local_rank):
-    w = W.decode_workload()
+    w = W.decode_workload(args.decode_batch)
     if args.impl == "reference":
         if rank != 0:
             return
@@ -499,10 +507,12 @@ def main_decode(args, rank, world, local_rank):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak,
+                         "traffic": recorded_traffic(w.name, "attn_decode", DECODE_SOURCES)
+                         if splits == 1 else None,
                          "peak_source": f"{src} hbm_gbs (copy)" if src == "measured"
                          else "fallback 6650 GB/s",
-                         "kernel": "attn_decode_split<128,4>"
+                         "kernel": "attn_decode_tma<128,3>"
                                    + (" + attn_decode_combine<128>" if splits > 1 else ""),
                          "timed_as": "whole attn_decode call (both kernels)"},
             "clocks": clocks,
@@ -599,6 +609,8 @@ def main():
     ap.add_argument("--workload", default="3", choices=["1", "2", "3", "4", "5", "decode"])
     ap.add_argument("--splits", type=int, default=0,
                     help="decode only: cache slices (0 = attn_decode_default_splits)")
+    ap.add_argument("--decode-batch", type=int, default=64,
+                    help="decode only: sequences (64 is the benchmark; smaller for profiling)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

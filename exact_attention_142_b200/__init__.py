@@ -6,7 +6,7 @@ binding over it.  ``attention`` is a convenience wrapper that allocates the
 outputs with torch and calls ``attn_fwd``.
 """
 from ._binding import (  # noqa: F401
-    ATTN_ERR_ALIGN, ATTN_ERR_CUDA, ATTN_ERR_DEVICE_TIMEOUT, ATTN_ERR_NULL, ATTN_ERR_SCALE,
+    ATTN_ERR_ALIGN, ATTN_ERR_CUDA, ATTN_ERR_DEVICE_TIMEOUT, ATTN_ERR_NULL, ATTN_ERR_PAGE, ATTN_ERR_SCALE,
     ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WINDOW, ATTN_ERR_WORKSPACE, ATTN_OK, AttnError,
     attn_decode, attn_decode_default_splits, attn_decode_workspace_bytes, attn_device_status,
     attn_fwd, attn_fwd_host, attn_fwd_host_workspace_bytes,
@@ -66,6 +66,6 @@ def attention_with_kvcache(q, k_cache, v_cache, cache_seqlens, *, block_table=No
     nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, page_size, pages_per_seq, num_splits)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
     attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq, d,
-                page_size, pages_per_seq, scale, causal, window_left, window_right, num_splits,
-                ws, nbytes, stream)
+                page_size, pages_per_seq, k_cache.shape[0], scale, causal, window_left,
+                window_right, num_splits, ws, nbytes, stream)
     return o, lse

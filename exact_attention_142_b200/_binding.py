@@ -25,6 +25,7 @@ ATTN_ERR_CUDA = -6
 ATTN_ERR_SCALE = -7
 ATTN_ERR_WORKSPACE = -8
 ATTN_ERR_DEVICE_TIMEOUT = -9
+ATTN_ERR_PAGE = -10
 
 
 class AttnError(RuntimeError):
@@ -58,8 +59,8 @@ def load_library():
         lib.attn_fwd_host_workspace_bytes.restype = S
         lib.attn_fwd_host_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.attn_decode.restype = I
-        lib.attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, I, I, I, P, S,
-                                    P]
+        lib.attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, I, I, P,
+                                    S, P]
         lib.attn_decode_workspace_bytes.restype = S
         lib.attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
         lib.attn_decode_default_splits.restype = I
@@ -127,14 +128,15 @@ def attn_fwd_host(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window
 
 
 def attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq, d,
-                page_size, pages_per_seq, scale, causal=True, window_left=-1, window_right=-1,
-                num_splits=1, workspace=None, workspace_bytes=0, stream=None,
+                page_size, pages_per_seq, num_pages, scale, causal=True, window_left=-1,
+                window_right=-1, num_splits=1, workspace=None, workspace_bytes=0, stream=None,
                 check=True) -> int:
     """Enqueue the key/value-cache decode on device buffers (see include/attn.h)."""
     lib = load_library()
     rc = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
                          _ptr(cache_seqlens), _ptr(block_table), int(B), int(Hq), int(Hkv),
-                         int(Nq), int(d), int(page_size), int(pages_per_seq), float(scale),
+                         int(Nq), int(d), int(page_size), int(pages_per_seq), int(num_pages),
+                         float(scale),
                          int(bool(causal)), int(window_left), int(window_right), int(num_splits),
                          _ptr(workspace), int(workspace_bytes), _stream(stream))
     if check and rc != ATTN_OK:

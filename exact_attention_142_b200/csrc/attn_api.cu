@@ -11,6 +11,7 @@
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_internal.h"
 
 namespace {
 
@@ -248,6 +249,7 @@ extern "C" const char* attn_status_string(int status) {
         case ATTN_ERR_SCALE: return "scale must be finite and > 0";
         case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out; outputs are undefined";
+        case ATTN_ERR_PAGE: return "a page-table entry lies outside the cache; outputs are undefined";
         default: return "unknown status";
     }
 }
@@ -257,7 +259,9 @@ extern "C" int attn_device_status(void) {
     if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
     const int zero = 0;
     if (cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
-    return v;
+    int dv = 0;
+    if (attn::decode_status_take(&dv) != ATTN_OK) return ATTN_ERR_CUDA;
+    return v != ATTN_OK ? v : dv;
 }
 
 extern "C" int attn_selftest_bounded_wait(uint64_t limit_ns, struct CUstream_st* stream) {

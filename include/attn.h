@@ -52,8 +52,10 @@ enum attn_status {
     ATTN_ERR_CUDA = -6,          /* a CUDA runtime / driver call failed               */
     ATTN_ERR_SCALE = -7,         /* scale is not a finite number > 0                  */
     ATTN_ERR_WORKSPACE = -8,     /* attn_fwd_host: workspace missing or too small     */
-    ATTN_ERR_DEVICE_TIMEOUT = -9 /* reported by attn_device_status(): a kernel wait
-                                    ran past its time limit and the kernel gave up   */
+    ATTN_ERR_DEVICE_TIMEOUT = -9, /* reported by attn_device_status(): a kernel wait
+                                     ran past its time limit and the kernel gave up  */
+    ATTN_ERR_PAGE = -10          /* reported by attn_device_status(): attn_decode met a
+                                    page-table entry outside [0, num_pages)          */
 };
 
 /*
@@ -110,51 +112,64 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
 /*
  * attn_decode -- attention of the newest tokens against a key/value cache,
  * split along the cache ("FlashAttention" explainer page, How it works, Step 9:
- * decoding with a cache of past keys and values; the split partials are merged
- * by the online-softmax rule of "Long context beyond a single GPU").
+ * decoding with a cache of past keys and values; the slices' partial results
+ * are merged by the online-softmax rescaling; paged layouts: "Use the decoding
+ * kernels for serving").
  *
  *   q       [B, Nq, Hq, d] bf16: the Nq (1..16) newest tokens of each sequence
- *   k_cache, v_cache [num_pages, page_size, Hkv, d] bf16 (paged cache)
+ *   k_cache, v_cache [num_pages, page_size, Hkv, d] bf16 (a pool of pages)
  *   block_table  device int32 [B, pages_per_seq]: page of logical page p of
  *           sequence b; NULL means page b * pages_per_seq + p, i.e. a contiguous
- *           cache [B, pages_per_seq * page_size, Hkv, d].
+ *           cache [B, pages_per_seq * page_size, Hkv, d] (num_pages must then
+ *           be >= B * pages_per_seq).  Entries for pages past a sequence's
+ *           length are never read.  An entry outside [0, num_pages) is not
+ *           followed: attn_device_status() then reports ATTN_ERR_PAGE.
  *   cache_seqlens device int32 [B]: keys held by sequence b, the new tokens
  *           included (Nq <= cache_seqlens[b] <= page_size * pages_per_seq).
+ *           Cached keys and values at positions below that length must be
+ *           finite; slots past it are never used, whatever they hold.
  *   o       [B, Nq, Hq, d] bf16;  lse [B, Hq, Nq] fp32 (natural log).
  * Query row i of sequence b sits at position pos = cache_seqlens[b] - Nq + i;
  * key j is visible iff (window_left < 0 || j >= pos - window_left) &&
  * (window_right < 0 || j <= pos + window_right), causal forcing window_right = 0.
+ *   page_size: any >= 1; a multiple of 8 (or a contiguous cache) takes the
+ *           TMA / tensor-core kernel, other sizes a slower gather kernel.
  *   num_splits: number of slices of the cache (>= 1; see
  *           attn_decode_default_splits).  With more than one slice, partial
  *           results go to `workspace` (device, 256-byte aligned, at least
  *           attn_decode_workspace_bytes(...) bytes; may be NULL when that is 0).
  * Asynchronous on `stream`; allocates nothing.  The host never reads
  * cache_seqlens or block_table; their contents are the caller's responsibility.
- * Returns ATTN_OK or a negative attn_status (ATTN_ERR_UNSUPPORTED for Nq > 16).
+ * Returns ATTN_OK or a negative attn_status (ATTN_ERR_UNSUPPORTED for Nq > 16,
+ * ATTN_ERR_SHAPE when num_pages * page_size exceeds 2^31 - 1).
  */
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                 const int32_t* cache_seqlens, const int32_t* block_table, int B, int Hq, int Hkv,
-                int Nq, int d, int page_size, int pages_per_seq, float scale, int causal,
-                int window_left, int window_right, int num_splits, void* workspace,
+                int Nq, int d, int page_size, int pages_per_seq, int num_pages, float scale,
+                int causal, int window_left, int window_right, int num_splits, void* workspace,
                 size_t workspace_bytes, struct CUstream_st* stream);
 
 /* Device workspace attn_decode needs for these sizes (0 when one slice). */
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int page_size,
                                    int pages_per_seq, int num_splits);
 
-/* A slice count that gives about four CTAs per SM, with at least 256 keys per
- * slice (max_cache_len = page_size * pages_per_seq). */
+/* A slice count for these sizes: the smallest that occupies at least half of
+ * the current device's CTA slots (two per SM) with a last wave at least half
+ * full (or at least four waves), keeping >= 256 keys per slice
+ * (max_cache_len = page_size * pages_per_seq).  Without a device it assumes
+ * 148 SMs. */
 int attn_decode_default_splits(int B, int Hq, int Hkv, int Nq, int max_cache_len);
 
 /* Static text for a status code (never NULL). */
 const char* attn_status_string(int status);
 
 /*
- * attn_device_status -- read and clear the status word of the current device.
- * Call after synchronising the streams that ran attn_fwd.  Returns ATTN_OK,
- * ATTN_ERR_DEVICE_TIMEOUT if any kernel since the last call gave up on a
- * bounded wait (its outputs are then undefined), or ATTN_ERR_CUDA if the word
- * could not be read.
+ * attn_device_status -- read and clear the status words of the current device.
+ * Call after synchronising the streams that ran attn_fwd / attn_decode.
+ * Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT if any kernel since the last call
+ * gave up on a bounded wait, ATTN_ERR_PAGE if attn_decode met a page-table
+ * entry outside the cache (the outputs of that call are then undefined), or
+ * ATTN_ERR_CUDA if a word could not be read.
  */
 int attn_device_status(void);
 

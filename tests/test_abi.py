@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, -10, -1):
+    for code in range(0, -11, -1):
         s = ea.attn_status_string(code)
         assert s and s != "unknown status", code
     assert ea.attn_status_string(-1234) == "unknown status"
@@ -111,7 +111,7 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 def call_decode(**over):
     args = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, o=FAKE, lse=FAKE, cache_seqlens=FAKE,
                 block_table=None, B=2, Hq=8, Hkv=2, Nq=1, d=128, page_size=16, pages_per_seq=8,
-                scale=0.1, causal=1, window_left=-1, window_right=-1, num_splits=1,
+                num_pages=16, scale=0.1, causal=1, window_left=-1, window_right=-1, num_splits=1,
                 workspace=None, workspace_bytes=0, stream=0)
     args.update(over)
     return ea.attn_decode(check=False, **args)
@@ -125,6 +125,9 @@ def call_decode(**over):
     (dict(pages_per_seq=0), ea.ATTN_ERR_SHAPE),
     (dict(num_splits=0), ea.ATTN_ERR_SHAPE),
     (dict(page_size=1 << 20, pages_per_seq=1 << 12), ea.ATTN_ERR_SHAPE),  # > 2^31 keys
+    (dict(num_pages=0), ea.ATTN_ERR_SHAPE),
+    (dict(num_pages=15), ea.ATTN_ERR_SHAPE),              # contiguous cache needs B * pps pages
+    (dict(num_pages=1 << 28, block_table=FAKE), ea.ATTN_ERR_SHAPE),  # rows overflow int32
     (dict(window_left=-3), ea.ATTN_ERR_WINDOW),
     (dict(d=80), ea.ATTN_ERR_UNSUPPORTED),
     (dict(Nq=17), ea.ATTN_ERR_UNSUPPORTED),
@@ -156,10 +159,14 @@ def test_decode_workspace_size(lib):
 
 
 def test_decode_default_splits(lib):
-    # few sequences and a long cache: many slices, at least 256 keys each
-    s = ea.attn_decode_default_splits(1, 32, 8, 1, 8192)
-    assert 8 <= s <= 32
+    # no device here: 148 SMs x 2 CTAs = 296 slots
+    # 64 sequences x 8 kv heads = 512 CTAs: 1.73 waves, last wave 216 >= 148 -> 1 slice
+    assert ea.attn_decode_default_splits(64, 32, 8, 1, 8192) == 1
+    # one sequence, 8 kv heads: 19 slices = 152 CTAs >= 148 slots
+    assert ea.attn_decode_default_splits(1, 32, 8, 1, 8192) == 19
+    # a short cache caps the slices (>= 256 keys each)
     assert ea.attn_decode_default_splits(1, 32, 8, 1, 300) == 1
-    # enough sequences to fill the GPU: one or two slices
-    assert ea.attn_decode_default_splits(256, 32, 8, 1, 8192) == 1
+    assert ea.attn_decode_default_splits(1, 32, 8, 1, 2048) == 8
+    # 300 CTAs: last waves of 4, 8, 12 CTAs are too small; 4 slices = 4.05 waves
+    assert ea.attn_decode_default_splits(75, 32, 4, 1, 8192) == 4
     assert ea.attn_decode_default_splits(0, 32, 8, 1, 8192) == 1

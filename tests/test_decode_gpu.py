@@ -33,8 +33,8 @@ def run_gpu(w: W.DecodeWorkload, q, kc, vc, seqlens, table, num_splits, *, q_dev
                                             w.pages_per_seq, num_splits)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=DEV)
     ea.attn_decode(qd, kd, vd, o, lse, sd, td, w.B, w.Hq, w.Hkv, w.Nq, w.d, w.page_size,
-                   w.pages_per_seq, w.scale, w.causal, w.window_left, w.window_right,
-                   num_splits, ws if nbytes else None, nbytes)
+                   w.pages_per_seq, kd.shape[0], w.scale, w.causal, w.window_left,
+                   w.window_right, num_splits, ws if nbytes else None, nbytes)
     torch.cuda.synchronize()
     assert ea.attn_device_status() == ea.ATTN_OK
     return o.cpu(), lse.cpu()
@@ -76,7 +76,11 @@ CASES = [
     case("nq16_mha_d128", 2, 2, 2, 16, 128, 128, 4, [16, 500]),
     case("gqa4_nq1_d64", 3, 8, 2, 1, 64, 16, 40, [64, 65, 639]),
     case("gqa8_nq2_d64", 2, 32, 4, 2, 64, 64, 10, [100, 640]),
-    case("odd_page7_d128", 2, 8, 2, 2, 128, 7, 50, [349, 350]),
+    case("odd_page7_d128", 2, 8, 2, 2, 128, 7, 50, [349, 350]),       # gather kernel
+    case("page100_d64", 2, 8, 2, 1, 64, 100, 6, [599, 301]),          # gather kernel
+    case("page1_d128", 2, 4, 2, 2, 128, 1, 150, [150, 77]),            # gather kernel
+    case("page24_d128", 2, 8, 2, 2, 128, 24, 30, [700, 31]),          # 8-key TMA copies
+    case("page256_d128", 2, 8, 1, 1, 128, 256, 3, [700, 256]),        # 64-key copies
     case("contiguous_d128", 3, 8, 2, 2, 128, 64, 8, [2, 300, 512], paged=False),
     case("window_causal_d128", 2, 8, 2, 4, 128, 32, 20, [640, 200], left=100),
     case("window_noncausal_d64", 2, 8, 2, 4, 64, 32, 20, [640, 37], causal=False, left=50,
@@ -137,8 +141,7 @@ def test_split_counts_agree():
                                                (200, False, -1), (5, False, 3)])
 def test_mask_pattern_bit_exact(left, causal, right):
     """Q = 0 makes every visible score 0, so exp(LSE) is the number of visible
-    keys; with V = one-hot of (key index mod d) the output's support shows
-    which residues were visible."""
+    keys, which must equal the oracle's count for every row."""
     w = case("mask", 2, 4, 2, 5, 128, 16, 30, [470, 5], causal=causal, left=left, right=right)
     q, kc, vc, seqlens, table = W.decode_inputs(w)
     q.zero_()
@@ -172,3 +175,25 @@ def test_benchmark_workload_sampled():
     qc, kcc, vcc = q.cpu(), kc.cpu(), vc.cpu()
     o_ref, lse_ref, _ = run_oracle(sub, qc[pick], kcc, vcc, seqlens[pick], table[pick])
     compare(o[pick], lse[pick], o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("page_size", [32, 7])
+def test_invalid_page_is_reported_not_followed(page_size):
+    """A page-table entry outside [0, num_pages) is neither read nor followed:
+    the call completes and attn_device_status reports ATTN_ERR_PAGE once."""
+    w = case("badpage", 2, 8, 2, 1, 128, page_size, 10, [5 * page_size, 2 * page_size])
+    q, kc, vc, seqlens, table = W.decode_inputs(w)
+    bad = table.clone()
+    bad[0, 1] = kc.shape[0] + 5
+    bad[1, 0] = -3
+    qd, kd, vd = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=DEV)
+    ea.attn_decode(qd, kd, vd, o, lse, seqlens.to(DEV), bad.to(DEV), w.B, w.Hq, w.Hkv, w.Nq, w.d,
+                   w.page_size, w.pages_per_seq, kd.shape[0], w.scale, True, -1, -1, 1)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_ERR_PAGE
+    assert ea.attn_device_status() == ea.ATTN_OK  # read clears it
+    # the context still works: a valid call afterwards matches the oracle
+    o_ref, lse_ref, _ = run_oracle(w, q, kc, vc, seqlens, table)
+    compare(*run_gpu(w, q, kc, vc, seqlens, table, 2), o_ref, lse_ref)

@@ -165,12 +165,14 @@ class DecodeWorkload:
         return self.page_size * self.pages_per_seq
 
 
-def decode_workload() -> DecodeWorkload:
-    """The decode benchmark: 64 sequences, each with a full 8192-token cache,
-    one new token, the grouped-query head layout of the 8192-token causal
-    workload (32 query heads over 8 key/value heads, d = 128), 64-token pages."""
-    return DecodeWorkload("decode_gqa_b64_hq32_hkv8_l8192_d128_page64", 64, 32, 8, 1, 128, 64, 128,
-                          [8192] * 64, True, True, -1, -1, 5)
+def decode_workload(B: int = 64) -> DecodeWorkload:
+    """The decode benchmark: B (64) sequences, each with a full 8192-token
+    cache, one new token, the grouped-query head layout of the 8192-token
+    causal workload (32 query heads over 8 key/value heads, d = 128), 64-token
+    pages.  Smaller B gives the same shape at a smaller size (B = 8: 268 MB of
+    cache, still twice the L2)."""
+    return DecodeWorkload(f"decode_gqa_b{B}_hq32_hkv8_l8192_d128_page64", B, 32, 8, 1, 128, 64,
+                          128, [8192] * B, True, True, -1, -1, 5)
 
 
 def decode_inputs(w: DecodeWorkload, device: str = "cpu"):
