@@ -61,6 +61,9 @@ def load_library():
         lib.attn_decode.restype = I
         lib.attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, I, I, P,
                                     S, P]
+        lib.attn_decode_noalloc.restype = I
+        lib.attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,
+                                            I, I, P]
         lib.attn_decode_workspace_bytes.restype = S
         lib.attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
         lib.attn_decode_default_splits.restype = I
@@ -141,6 +144,28 @@ def attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, 
                          _ptr(workspace), int(workspace_bytes), _stream(stream))
     if check and rc != ATTN_OK:
         raise AttnError(rc, "attn_decode")
+    return rc
+
+
+ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq,
+                        d, page_size, pages_per_seq, num_pages, scale, causal=True,
+                        window_left=-1, window_right=-1, num_splits=1, stream=None,
+                        check=True) -> int:
+    """attn_decode with the library's fixed scratch instead of a workspace, for
+    callers that must not allocate device memory while they run (see
+    include/attn.h)."""
+    lib = load_library()
+    rc = lib.attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                 _ptr(cache_seqlens), _ptr(block_table), int(B), int(Hq),
+                                 int(Hkv), int(Nq), int(d), int(page_size), int(pages_per_seq),
+                                 int(num_pages), float(scale), int(bool(causal)),
+                                 int(window_left), int(window_right), int(num_splits),
+                                 _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_decode_noalloc")
     return rc
 
 

@@ -290,3 +290,60 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
     return d == 128 ? launch_decode<128>(p, plan.rows, tma, s)
                     : launch_decode<64>(p, plan.rows, tma, s);
 }
+
+// ------------------------------------------------- decode without allocation
+// attn_decode_noalloc is attn_decode for callers that must not allocate device
+// memory while they run: a serving loop that commits nearly all of HBM to its
+// key/value page pool at start-up and keeps a fixed footprint afterwards, or a
+// latency-bound step loop, where cudaMalloc / cudaFree (which can block on and
+// synchronise with the device, and fail when the pool holds the memory) or a
+// framework allocator would stall or fail the step.  The slice partials live in
+// the fixed array below instead of a caller-provided workspace.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices];  // device address of the array, per device
+std::mutex g_noalloc_mu;
+
+// The array's address on the current device, looked up once per device (on the
+// first call that needs it, with that device current).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                   void* o, float* lse, const int32_t* cache_seqlens,
+                                   const int32_t* block_table, int B, int Hq, int Hkv, int Nq,
+                                   int d, int page_size, int pages_per_seq, int num_pages,
+                                   float scale, int causal, int window_left, int window_right,
+                                   int num_splits, struct CUstream_st* stream) {
+    // Host arithmetic only: 0 for a single slice (no scratch) or invalid sizes,
+    // which attn_decode then rejects with its own status.
+    const size_t need = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, page_size, pages_per_seq,
+                                                    num_splits);
+    if (need > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (need > 0) {
+        const int rc = noalloc_scratch(&scratch);
+        if (rc != ATTN_OK) return rc;
+    }
+    // Every scratch entry the merge kernel reads is written by the slice kernel
+    // of the same call, so nothing left by an earlier call needs clearing.
+    return attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq, d,
+                       page_size, pages_per_seq, num_pages, scale, causal, window_left,
+                       window_right, num_splits, scratch,
+                       need > 0 ? (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES : 0, stream);
+}

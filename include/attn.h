@@ -149,6 +149,35 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
                 int causal, int window_left, int window_right, int num_splits, void* workspace,
                 size_t workspace_bytes, struct CUstream_st* stream);
 
+/*
+ * attn_decode_noalloc -- attn_decode without a workspace argument and without
+ * allocating anything.  The pages have no counterpart to this entry point: it
+ * exists for callers that must not allocate device memory while they run, such
+ * as a serving loop that gives nearly all of HBM to its key/value page pool at
+ * start-up, or a latency-bound decode step, where cudaMalloc / cudaFree (which
+ * can block on and synchronise with the device, and fail once the pool holds
+ * the memory) or a framework allocator would stall or fail the step.
+ *
+ * Arguments and result are those of attn_decode.  The slice partials go to one
+ * fixed device array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES (8 MiB) inside the
+ * library, per device; a call whose attn_decode_workspace_bytes(...) exceeds
+ * that returns ATTN_ERR_WORKSPACE before doing anything (use fewer slices, or
+ * attn_decode with a workspace).  A single slice uses no scratch at all.
+ *
+ * The first call on a device that needs the scratch looks up the array's
+ * address (cudaGetSymbolAddress, with that device current) and keeps it; make
+ * that first call before any stream capture.  All calls on a device share the
+ * one array and it keeps the last call's contents (nothing in it needs to
+ * start at zero): calls that may overlap on the GPU -- other streams, other
+ * host threads -- race on it, so order them on one stream.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
+                        float* lse, const int32_t* cache_seqlens, const int32_t* block_table,
+                        int B, int Hq, int Hkv, int Nq, int d, int page_size, int pages_per_seq,
+                        int num_pages, float scale, int causal, int window_left, int window_right,
+                        int num_splits, struct CUstream_st* stream);
+
 /* Device workspace attn_decode needs for these sizes (0 when one slice). */
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int page_size,
                                    int pages_per_seq, int num_splits);
