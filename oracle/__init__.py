@@ -63,6 +63,15 @@ def load(path: Optional[str] = None):
         ctypes.c_int, ctypes.c_int, ctypes.c_double,  # page_size pages_per_seq scale
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,  # causal left right threads
     ]
+    lib.oracle_attn_bwd.restype = ctypes.c_int
+    lib.oracle_attn_bwd.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # q k v dout
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # dq dk dv
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,  # B Hq Hkv N d
+        ctypes.c_double,  # scale
+        ctypes.c_int, ctypes.c_int, ctypes.c_int,  # causal left right
+        ctypes.c_void_p, ctypes.c_int,  # cu_seqlens threads
+    ]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -151,3 +160,31 @@ def attn_kvcache(q, k_cache, v_cache, cache_seqlens, *, B: int, Hq: int, Hkv: in
     if rc != 0:
         raise ValueError(f"oracle_attn_kvcache failed with code {rc}")
     return o, lse, nvis
+
+
+def attn_bwd(q, k, v, dout, *, B: int, Hq: int, Hkv: int, N: int, d: int, scale: float,
+             causal: bool = False, window_left: int = -1, window_right: int = -1,
+             cu_seqlens: Optional[Sequence[int]] = None, nthreads: int = 0, lib=None):
+    """Gradients of sum(dout * O) with respect to q, k, v.
+
+    q, dout [tokens, Hq, d] (or [B, N, Hq, d]) bf16 bits; k, v [tokens, Hkv, d].
+    Returns fp64 (dq [tokens, Hq, d], dk [tokens, Hkv, d], dv [tokens, Hkv, d]).
+    """
+    lib = lib or load()
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        tokens = int(cu[-1])
+    else:
+        tokens = B * N
+    dq = np.empty((tokens, Hq, d), dtype=np.float64)
+    dk = np.empty((tokens, Hkv, d), dtype=np.float64)
+    dv = np.empty((tokens, Hkv, d), dtype=np.float64)
+    rc = lib.oracle_attn_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data,
+                             dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, B, Hq, Hkv, N, d,
+                             float(scale), int(bool(causal)), int(window_left), int(window_right),
+                             None if cu is None else cu.ctypes.data, int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd failed with code {rc}")
+    return dq, dk, dv

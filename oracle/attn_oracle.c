@@ -336,3 +336,172 @@ int oracle_attn_kvcache(const uint16_t *q, const uint16_t *kc, const uint16_t *v
     }
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/*
+ * oracle_attn_bwd -- gradients of attention with respect to q, k and v.
+ *
+ * The pages ("FlashAttention" explainer page, How it works, Step 5, and
+ * "Backward pass in a bit more detail") say what the backward pass needs
+ * (queries, keys, values, the output gradient and each row's log-sum-exp; the
+ * weights are rebuilt, key/value gradients accumulate over query rows and
+ * query gradients over keys) but print no formulas.  This is the plain
+ * chain rule for L = sum(dO * O) with O the forward above:
+ *   P_ij  = exp(s_ij - LSE_i)              (the forward's weights)
+ *   dP_ij = dO_i . v_j
+ *   D_i   = sum_j P_ij dP_ij
+ *   dS_ij = P_ij (dP_ij - D_i)             (softmax Jacobian)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i        summed over the query heads of the group
+ *   dV_j  = sum_i P_ij dO_i                summed over the query heads of the group
+ * with the forward's masks, head groups and sequences.  Phase 1 walks query
+ * rows (scores, LSE, D and dQ); phase 2 walks keys and rebuilds the weights of
+ * every row that sees the key from the row's LSE and D.
+ *   q, dout [tokens, Hq, d] bf16 bits;  k, v [tokens, Hkv, d] bf16 bits
+ *   dq [tokens, Hq, d] fp64;  dk, dv [tokens, Hkv, d] fp64
+ * A row with no visible key contributes nothing.
+ */
+static double dot_bf16(const uint16_t *a, const uint16_t *b, int d) {
+    double s = 0.0;
+    for (int t = 0; t < d; ++t) s += widen_bf16(a[t]) * widen_bf16(b[t]);
+    return s;
+}
+
+int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    const uint16_t *dout, double *dq, double *dk, double *dv,
+                    int B, int Hq, int Hkv, int N, int d, double scale,
+                    int causal, int window_left, int window_right,
+                    const int32_t *cu_seqlens, int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0) return ORACLE_ERR_ARG;
+    if (Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    if (window_left < -1 || window_right < -1) return ORACLE_ERR_ARG;
+    const int group = Hq / Hkv;
+    const int64_t left = window_left;
+    const int64_t right = causal ? 0 : window_right;
+    const int64_t tokens = cu_seqlens ? (int64_t)cu_seqlens[B] : (int64_t)B * N;
+    int64_t maxL = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t L = cu_seqlens ? (int64_t)cu_seqlens[b + 1] - cu_seqlens[b] : N;
+        if (L < 0) return ORACLE_ERR_ARG;
+        if (L > maxL) maxL = L;
+    }
+#ifdef _OPENMP
+    const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#else
+    (void)nthreads;
+#endif
+    double *lse = (double *)malloc(sizeof(double) * (size_t)(tokens * Hq > 0 ? tokens * Hq : 1));
+    double *D = (double *)malloc(sizeof(double) * (size_t)(tokens * Hq > 0 ? tokens * Hq : 1));
+    if (!lse || !D) {
+        free(lse);
+        free(D);
+        return ORACLE_ERR_NOMEM;
+    }
+    int failed = 0;
+
+    /* Phase 1: one query row at a time -- LSE_i, D_i and dQ_i. */
+#pragma omp parallel num_threads(nt)
+    {
+        double *s_row = (double *)malloc(sizeof(double) * (size_t)(maxL > 0 ? maxL : 1));
+        double *dp_row = (double *)malloc(sizeof(double) * (size_t)(maxL > 0 ? maxL : 1));
+        if (!s_row || !dp_row) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t u = 0; u < tokens * Hq; ++u) {
+            if (!s_row || !dp_row) continue;
+            const int64_t t = u / Hq;
+            const int h = (int)(u % Hq), g = h / group;
+            int b = 0;
+            if (cu_seqlens) {
+                while (b + 1 < B && cu_seqlens[b + 1] <= t) ++b;
+            } else {
+                b = (int)(t / (N > 0 ? N : 1));
+            }
+            const int64_t start = cu_seqlens ? cu_seqlens[b] : (int64_t)b * N;
+            const int64_t L = cu_seqlens ? (int64_t)cu_seqlens[b + 1] - cu_seqlens[b] : N;
+            const int64_t i = t - start;
+            const uint16_t *qi = q + (t * Hq + h) * (int64_t)d;
+            const uint16_t *doi = dout + (t * Hq + h) * (int64_t)d;
+            double *dqi = dq + (t * Hq + h) * (int64_t)d;
+            for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+            double M = -INFINITY;
+            int64_t nvis = 0;
+            for (int64_t j = 0; j < L; ++j) {
+                if (!key_visible(i, j, left, right)) {
+                    s_row[j] = -INFINITY;
+                    continue;
+                }
+                const int64_t kj = ((start + j) * Hkv + g) * (int64_t)d;
+                s_row[j] = scale * dot_bf16(qi, k + kj, d);
+                dp_row[j] = dot_bf16(doi, v + kj, d);
+                if (s_row[j] > M) M = s_row[j];
+                ++nvis;
+            }
+            if (nvis == 0) {
+                lse[u] = -INFINITY;
+                D[u] = 0.0;
+                continue;
+            }
+            double Z = 0.0;
+            for (int64_t j = 0; j < L; ++j)
+                if (s_row[j] != -INFINITY) Z += exp(s_row[j] - M);
+            const double lse_i = M + log(Z);
+            double Di = 0.0;
+            for (int64_t j = 0; j < L; ++j)
+                if (s_row[j] != -INFINITY) Di += exp(s_row[j] - lse_i) * dp_row[j];
+            lse[u] = lse_i;
+            D[u] = Di;
+            for (int64_t j = 0; j < L; ++j) {
+                if (s_row[j] == -INFINITY) continue;
+                const double ds = exp(s_row[j] - lse_i) * (dp_row[j] - Di);
+                const uint16_t *kj = k + ((start + j) * Hkv + g) * (int64_t)d;
+                for (int c = 0; c < d; ++c) dqi[c] += scale * ds * widen_bf16(kj[c]);
+            }
+        }
+        free(s_row);
+        free(dp_row);
+    }
+
+    /* Phase 2: one key at a time -- dK_j and dV_j over every row that sees it. */
+    if (!failed) {
+#pragma omp parallel for schedule(dynamic, 16) num_threads(nt)
+        for (int64_t u = 0; u < tokens * Hkv; ++u) {
+            const int64_t t = u / Hkv;
+            const int g = (int)(u % Hkv);
+            int b = 0;
+            if (cu_seqlens) {
+                while (b + 1 < B && cu_seqlens[b + 1] <= t) ++b;
+            } else {
+                b = (int)(t / (N > 0 ? N : 1));
+            }
+            const int64_t start = cu_seqlens ? cu_seqlens[b] : (int64_t)b * N;
+            const int64_t L = cu_seqlens ? (int64_t)cu_seqlens[b + 1] - cu_seqlens[b] : N;
+            const int64_t j = t - start;
+            const uint16_t *kj = k + (t * Hkv + g) * (int64_t)d;
+            const uint16_t *vj = v + (t * Hkv + g) * (int64_t)d;
+            double *dkj = dk + (t * Hkv + g) * (int64_t)d;
+            double *dvj = dv + (t * Hkv + g) * (int64_t)d;
+            for (int c = 0; c < d; ++c) dkj[c] = dvj[c] = 0.0;
+            for (int hh = 0; hh < group; ++hh) {
+                const int h = g * group + hh;
+                for (int64_t i = 0; i < L; ++i) {
+                    if (!key_visible(i, j, left, right)) continue;
+                    const int64_t r = (start + i) * Hq + h;
+                    const uint16_t *qi = q + r * (int64_t)d;
+                    const uint16_t *doi = dout + r * (int64_t)d;
+                    const double p = exp(scale * dot_bf16(qi, kj, d) - lse[r]);
+                    const double ds = p * (dot_bf16(doi, vj, d) - D[r]);
+                    for (int c = 0; c < d; ++c) {
+                        dkj[c] += scale * ds * widen_bf16(qi[c]);
+                        dvj[c] += p * widen_bf16(doi[c]);
+                    }
+                }
+            }
+        }
+    }
+    free(lse);
+    free(D);
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

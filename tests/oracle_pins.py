@@ -24,6 +24,11 @@ What pins what:
     float64 on the CPU with a band mask built by torch.triu / torch.tril (the
     page's own causal-mask recipe in "Checking correctness"), and
     torch.logsumexp for the LSE.
+  * gradients       -- central finite differences of sum(dO * O) computed by a
+    numpy forward written in the pin; torch autograd through float64
+    scaled_dot_product_attention; the zero-sum of key gradients and the
+    value-gradient sum; packed == separate; grouped == repeated with the
+    gradients summed.
 """
 from __future__ import annotations
 
@@ -503,6 +508,142 @@ def pin_kvcache_torch_sdpa(lib):
         assert np.abs(lse[b] - ref_lse).max() <= 1e-12
 
 
+# --------------------------------------------------------------------------
+# backward (gradients)
+# --------------------------------------------------------------------------
+def _bwd(lib, q, k, v, do, **kw):
+    return oracle.attn_bwd(W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v), W.bf16_bits(do),
+                           lib=lib, **kw)
+
+
+def _np_forward_loss(qf, kf, vf, dof, scale, visible):
+    """sum(dO * O) for one head, written out in numpy (fp64): the function
+    whose gradient the oracle must return."""
+    s = scale * qf @ kf.T
+    s = np.where(visible, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    e = np.where(visible, np.exp(s - m), 0.0)
+    o = (e / e.sum(axis=1, keepdims=True)) @ vf
+    return float((dof * o).sum())
+
+
+def pin_bwd_finite_differences(lib):
+    """Central differences of sum(dO * O), computed by a numpy forward, match
+    the oracle's gradients (independent of the oracle's formulas)."""
+    rng = np.random.default_rng(40)
+    for (N, d, causal, left, right, scale) in [(6, 4, True, -1, -1, 0.7),
+                                               (7, 3, False, 2, 1, 0.9),
+                                               (5, 4, False, -1, -1, 0.5)]:
+        q = _bf16(rng.standard_normal((1, N, 1, d)))
+        k = _bf16(rng.standard_normal((1, N, 1, d)))
+        v = _bf16(rng.standard_normal((1, N, 1, d)))
+        do = _bf16(rng.standard_normal((1, N, 1, d)))
+        dq, dk, dv = _bwd(lib, q, k, v, do, B=1, Hq=1, Hkv=1, N=N, d=d, scale=scale,
+                          causal=causal, window_left=left, window_right=right)
+        vis = _band_mask(N, causal, left, right).numpy()
+        base = [_f64(t).reshape(N, d) for t in (q, k, v, do)]
+        eps = 1e-6
+        for which, grad in ((0, dq), (1, dk), (2, dv)):
+            g = grad.reshape(N, d)
+            for i in range(N):
+                for c in range(d):
+                    plus = [a.copy() for a in base]
+                    minus = [a.copy() for a in base]
+                    plus[which][i, c] += eps
+                    minus[which][i, c] -= eps
+                    fd = (_np_forward_loss(*plus[:3], plus[3], scale, vis) -
+                          _np_forward_loss(*minus[:3], minus[3], scale, vis)) / (2 * eps)
+                    assert abs(fd - g[i, c]) <= 1e-6 * (1 + abs(fd)), (which, i, c, fd, g[i, c])
+
+
+def pin_bwd_torch_autograd(lib):
+    """torch autograd through float64 scaled_dot_product_attention with a band
+    mask, grouped heads summed back onto their key/value head."""
+    import torch.nn.functional as F
+    rng = np.random.default_rng(41)
+    cases = [
+        # B, N, Hq, Hkv, d, causal, left, right, scale
+        (2, 37, 4, 2, 16, True, -1, -1, 16 ** -0.5),
+        (1, 29, 3, 3, 8, False, 5, 2, 0.4),
+        (1, 41, 6, 1, 32, True, 9, 0, 32 ** -0.5),
+    ]
+    for (B, N, Hq, Hkv, d, causal, left, right, scale) in cases:
+        q = _bf16(rng.standard_normal((B, N, Hq, d)))
+        k = _bf16(rng.standard_normal((B, N, Hkv, d)))
+        v = _bf16(rng.standard_normal((B, N, Hkv, d)))
+        do = _bf16(rng.standard_normal((B, N, Hq, d)))
+        dq, dk, dv = _bwd(lib, q, k, v, do, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=scale,
+                          causal=causal, window_left=left, window_right=right)
+        g = Hq // Hkv
+        qt = q.to(torch.float64).requires_grad_()
+        kt = k.to(torch.float64).requires_grad_()
+        vt = v.to(torch.float64).requires_grad_()
+        kr = torch.repeat_interleave(kt, g, dim=2).transpose(1, 2)
+        vr = torch.repeat_interleave(vt, g, dim=2).transpose(1, 2)
+        o = F.scaled_dot_product_attention(qt.transpose(1, 2), kr, vr,
+                                           attn_mask=_band_mask(N, causal, left, right),
+                                           scale=scale).transpose(1, 2)
+        (o * do.to(torch.float64)).sum().backward()
+        for got, ref in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+            ref = ref.numpy().reshape(got.shape)
+            assert np.abs(got - ref).max() <= 1e-11 * (1 + np.abs(ref).max()), np.abs(got - ref).max()
+
+
+def pin_bwd_invariants(lib):
+    """Rows of dS sum to zero, so the key gradients of a sequence and head sum
+    to zero; rows of P sum to one, so the value gradients sum to the output
+    gradients of the rows that see any key."""
+    rng = np.random.default_rng(42)
+    lens = [13, 1, 22]
+    cu = W.cumulative(lens)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 8
+    q = _bf16(rng.standard_normal((T, Hq, d)))
+    k = _bf16(rng.standard_normal((T, Hkv, d)))
+    v = _bf16(rng.standard_normal((T, Hkv, d)))
+    do = _bf16(rng.standard_normal((T, Hq, d)))
+    for (causal, left, right) in [(True, -1, -1), (False, 3, 2), (True, 4, -1)]:
+        dq, dk, dv = _bwd(lib, q, k, v, do, B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=0.6,
+                          causal=causal, window_left=left, window_right=right, cu_seqlens=cu)
+        dof = _f64(do)
+        for b in range(3):
+            a, e = cu[b], cu[b + 1]
+            for gh in range(Hkv):
+                assert np.abs(dk[a:e, gh].sum(axis=0)).max() <= 1e-12
+                heads = range(gh * (Hq // Hkv), (gh + 1) * (Hq // Hkv))
+                want = sum(dof[a:e, h].sum(axis=0) for h in heads)
+                assert np.abs(dv[a:e, gh].sum(axis=0) - want).max() <= 1e-12
+
+
+def pin_bwd_packed_and_grouped(lib):
+    """A packed batch equals separate calls per sequence, and grouped heads
+    equal key/value heads repeated per query head with the gradients summed."""
+    rng = np.random.default_rng(43)
+    lens = [11, 4, 17]
+    cu = W.cumulative(lens)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 8
+    q = _bf16(rng.standard_normal((T, Hq, d)))
+    k = _bf16(rng.standard_normal((T, Hkv, d)))
+    v = _bf16(rng.standard_normal((T, Hkv, d)))
+    do = _bf16(rng.standard_normal((T, Hq, d)))
+    kw = dict(scale=0.45, causal=True, window_left=5)
+    dq, dk, dv = _bwd(lib, q, k, v, do, B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, cu_seqlens=cu, **kw)
+    for b, L in enumerate(lens):
+        a = cu[b]
+        sl = slice(a, a + L)
+        r = _bwd(lib, q[sl].unsqueeze(0).contiguous(), k[sl].unsqueeze(0).contiguous(),
+                 v[sl].unsqueeze(0).contiguous(), do[sl].unsqueeze(0).contiguous(), B=1, Hq=Hq,
+                 Hkv=Hkv, N=L, d=d, **kw)
+        for got, ref in zip((dq, dk, dv), r):
+            assert np.array_equal(got[sl], ref)
+    g = Hq // Hkv
+    kr = torch.repeat_interleave(k, g, dim=1).contiguous()
+    vr = torch.repeat_interleave(v, g, dim=1).contiguous()
+    dq2, dk2, dv2 = _bwd(lib, q, kr, vr, do, B=3, Hq=Hq, Hkv=Hq, N=T, d=d, cu_seqlens=cu, **kw)
+    assert np.abs(dq - dq2).max() <= 1e-12
+    assert np.abs(dk - dk2.reshape(T, Hkv, g, d).sum(axis=2)).max() <= 1e-12
+    assert np.abs(dv - dv2.reshape(T, Hkv, g, d).sum(axis=2)).max() <= 1e-12
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_uniform_scores,
@@ -521,4 +662,8 @@ ALL_PINS = [
     pin_kvcache_paged_equals_contiguous,
     pin_kvcache_uniform_closed_form,
     pin_kvcache_torch_sdpa,
+    pin_bwd_finite_differences,
+    pin_bwd_torch_autograd,
+    pin_bwd_invariants,
+    pin_bwd_packed_and_grouped,
 ]

@@ -34,6 +34,17 @@ MUTANTS = {
                                     "                        const int64_t page = 0\n                                                 ? block_table[(int64_t)b * pages_per_seq + j / page_size]"),
     "kvcache_page_row_swapped": ("const int64_t row = page * page_size + j % page_size;\n                        const uint16_t *vj",
                                  "const int64_t row = page * page_size + (page_size - 1 - j % page_size);\n                        const uint16_t *vj"),
+    "bwd_dq_scale_dropped": ("dqi[c] += scale * ds * widen_bf16(kj[c]);",
+                             "dqi[c] += ds * widen_bf16(kj[c]);"),
+    "bwd_D_not_subtracted": ("const double ds = exp(s_row[j] - lse_i) * (dp_row[j] - Di);",
+                             "const double ds = exp(s_row[j] - lse_i) * dp_row[j];"),
+    "bwd_dk_uses_k": ("dkj[c] += scale * ds * widen_bf16(qi[c]);",
+                      "dkj[c] += scale * ds * widen_bf16(kj[c]);"),
+    "bwd_dv_weight_dropped": ("dvj[c] += p * widen_bf16(doi[c]);", "dvj[c] += widen_bf16(doi[c]);"),
+    "bwd_group_sum_one_head": ("for (int hh = 0; hh < group; ++hh) {",
+                               "for (int hh = 0; hh < 1; ++hh) {"),
+    "bwd_key_mask_transposed": ("                    if (!key_visible(i, j, left, right)) continue;\n                    const int64_t r",
+                                "                    if (!key_visible(j, i, left, right)) continue;\n                    const int64_t r"),
 }
 
 
