@@ -8,7 +8,8 @@ outputs with torch and calls ``attn_fwd``.
 from ._binding import (  # noqa: F401
     ATTN_ERR_ALIGN, ATTN_ERR_CUDA, ATTN_ERR_DEVICE_TIMEOUT, ATTN_ERR_NULL, ATTN_ERR_PAGE, ATTN_ERR_SCALE,
     ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WINDOW, ATTN_ERR_WORKSPACE, ATTN_OK, AttnError,
-    ATTN_DECODE_NOALLOC_SCRATCH_BYTES, attn_decode, attn_decode_default_splits,
+    ATTN_DECODE_NOALLOC_SCRATCH_BYTES, attn_bwd, attn_bwd_workspace_bytes, attn_decode,
+    attn_decode_default_splits,
     attn_decode_noalloc, attn_decode_workspace_bytes, attn_device_status,
     attn_fwd, attn_fwd_host, attn_fwd_host_workspace_bytes,
     attn_selftest_bounded_wait, attn_status_string, library_path, load_library)

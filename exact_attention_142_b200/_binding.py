@@ -58,6 +58,10 @@ def load_library():
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P, S, P]
         lib.attn_fwd_host_workspace_bytes.restype = S
         lib.attn_fwd_host_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        lib.attn_bwd.restype = I
+        lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P, S, P]
+        lib.attn_bwd_workspace_bytes.restype = S
+        lib.attn_bwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.attn_decode.restype = I
         lib.attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, I, I, P,
                                     S, P]
@@ -128,6 +132,25 @@ def attn_fwd_host(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window
     if check and rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_host")
     return rc
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal=False,
+             window_left=-1, window_right=-1, cu_seqlens=None, max_seqlen=0, workspace=None,
+             workspace_bytes=0, stream=None, check=True) -> int:
+    """Enqueue the backward pass on device buffers (see include/attn.h)."""
+    lib = load_library()
+    rc = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                      _ptr(dv), int(B), int(Hq), int(Hkv), int(N), int(d), float(scale),
+                      int(bool(causal)), int(window_left), int(window_right), _ptr(cu_seqlens),
+                      int(max_seqlen), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd")
+    return rc
+
+
+def attn_bwd_workspace_bytes(B, Hq, Hkv, N, d, packed) -> int:
+    return int(load_library().attn_bwd_workspace_bytes(int(B), int(Hq), int(Hkv), int(N), int(d),
+                                                       int(bool(packed))))
 
 
 def attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq, d,

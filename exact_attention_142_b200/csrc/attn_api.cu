@@ -259,9 +259,10 @@ extern "C" int attn_device_status(void) {
     if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
     const int zero = 0;
     if (cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
-    int dv = 0;
+    int dv = 0, bv = 0;
     if (attn::decode_status_take(&dv) != ATTN_OK) return ATTN_ERR_CUDA;
-    return v != ATTN_OK ? v : dv;
+    if (attn::bwd_status_take(&bv) != ATTN_OK) return ATTN_ERR_CUDA;
+    return v != ATTN_OK ? v : (dv != ATTN_OK ? dv : bv);
 }
 
 extern "C" int attn_selftest_bounded_wait(uint64_t limit_ns, struct CUstream_st* stream) {

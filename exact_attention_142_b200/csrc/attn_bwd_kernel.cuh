@@ -1,0 +1,756 @@
+// attn_bwd_kernel.cuh -- gradients of exact attention for sm_100a.
+//
+// The backward pass recomputes the score tiles from Q and K and rebuilds the
+// weights from each row's saved log-sum-exp ("FlashAttention",
+// ozercemkelahmet.com/tools/flashattention, How it works, Step 5, and
+// "Backward pass in a bit more detail": key/value gradients accumulate over
+// query blocks, query gradients over key blocks).  With P_ij = exp(s_ij - LSE_i),
+// D_i = sum_c dO_ic O_ic and dS = P (dP - D):
+//
+//   attn_bwd_dsum    D_i for every (row, head), fp32, one warp per row.
+//   attn_bwd_dkv     one CTA per (sequence, key/value head, 128-key block).  K and
+//                    V stay in shared memory; the Q and dO tiles of every query
+//                    head of the group and every query block that sees the keys
+//                    stream through a 2-stage ring.  Per query block:
+//                      S^T = K Q^T, dP^T = V dO^T      (tcgen05, both from smem)
+//                      P^T, dS^T                        (8 warps, fp32 -> bf16)
+//                      dV += P^T dO, dK += dS^T Q       (A from tensor memory)
+//                    dK and dV stay in tensor memory for the whole loop, so each
+//                    key row is written once, already summed over the group.
+//   attn_bwd_dq      one CTA per (sequence, query head, 128-row block), over the
+//                    key blocks the rows see: S = Q K^T, dP = dO V^T, dS, then
+//                    dQ += dS K.  dQ stays in tensor memory; no atomics.
+//
+// Tensor memory (512 columns): dkv: S^T [0,128), dP^T [128,256), dV [256,256+d),
+// dK [384,384+d); dq: S [0,128), dP [128,256), dQ [256,256+d).  The bf16 P^T /
+// dS^T (dS) are written into the upper 64 columns of their fp32 source region
+// once both warpgroups have read it, and the next product reads them there.
+//
+// Warps: 0-7 elementwise (warpgroup x = warp / 4 takes the tile's columns
+// [64x, 64x + 64); warp w % 4 its 32 tensor-memory lanes), 8 TMA producer,
+// 9 MMA issuer (both converged, one elected lane issues).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "attn.h"
+#include "ptx.cuh"
+
+namespace attn {
+namespace bwd {
+
+// Device status word of the backward kernels (read by attn_device_status).
+__device__ int g_bwd_status;
+
+constexpr int kBM = 128;  // query rows per block
+constexpr int kBN = 128;  // keys per block
+constexpr int kThreads = 320;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr int kElemThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kBoxBytes = 128 * 128;  // one TMA box: 128 rows x 128 bytes
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+    const void* o;
+    const void* dout;
+    const float* lse;
+    float* dsum;  // D, laid out like lse
+    void* dq;
+    void* dk;
+    void* dv;
+    const int32_t* cu_seqlens;
+    int B, Hq, Hkv;
+    int N;         // dense: sequence length; packed: total tokens
+    int group;     // Hq / Hkv
+    int left, right;
+    int n_blocks;  // ceil(longest sequence / 128)
+    float scale;
+    float scale_log2;
+    unsigned long long wait_limit_ns;
+};
+
+// ------------------------------------------------------------ small helpers
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long limit_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (ptx::global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicCAS(&g_bwd_status, 0, ATTN_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::global_timer_ns() - t0 > limit_ns) {
+            atomicCAS(&g_bwd_status, 0, ATTN_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns) {
+    return __all_sync(0xffffffffu, bounded_wait(bar, parity, abort_flag, limit_ns));
+}
+
+__device__ __forceinline__ void elem_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kElemThreads) : "memory");
+}
+
+struct Seq {
+    int start, len;
+};
+
+__device__ __forceinline__ Seq seq_of(const BwdParams& p, int b) {
+    Seq s;
+    if (p.cu_seqlens) {
+        s.start = p.cu_seqlens[b];
+        s.len = p.cu_seqlens[b + 1] - s.start;
+    } else {
+        s.start = b * p.N;
+        s.len = p.N;
+    }
+    return s;
+}
+
+// Index of (sequence b, head h, row i) in lse / D: [B, Hq, N] dense, [Hq, T] packed.
+__device__ __forceinline__ size_t stat_index(const BwdParams& p, int b, int h, int start, int i) {
+    return p.cu_seqlens ? (size_t)h * p.N + start + i : ((size_t)b * p.Hq + h) * p.N + i;
+}
+
+__device__ __forceinline__ bool visible(const BwdParams& p, int q, int k) {
+    return (p.left < 0 || k >= q - p.left) && (p.right < 0 || k <= q + p.right);
+}
+
+// Every (query, key) pair of query block m x key block n is inside the
+// sequence and visible: no element mask needed.
+__device__ __forceinline__ bool block_full(const BwdParams& p, int m, int n, int len) {
+    const long long q0 = (long long)m * kBM, k0 = (long long)n * kBN;
+    if (q0 + kBM > len || k0 + kBN > len) return false;
+    if (p.left >= 0 && k0 < q0 + kBM - 1 - p.left) return false;
+    if (p.right >= 0 && k0 + kBN - 1 > q0 + p.right) return false;
+    return true;
+}
+
+// Query blocks [m_lo, m_hi) that see some key of key block n.
+__device__ __forceinline__ void query_blocks(const BwdParams& p, int n, int len, int& m_lo, int& m_hi) {
+    const long long k0 = (long long)n * kBN;
+    long long lo = p.right >= 0 ? k0 - p.right : 0;
+    long long hi = p.left >= 0 ? k0 + kBN + p.left : len;  // exclusive
+    if (lo < 0) lo = 0;
+    if (hi > len) hi = len;
+    m_lo = (int)(lo / kBM);
+    m_hi = hi > lo ? (int)((hi + kBM - 1) / kBM) : m_lo;
+}
+
+// Key blocks [n_lo, n_hi) that some row of query block m sees.
+__device__ __forceinline__ void key_blocks(const BwdParams& p, int m, int len, int& n_lo, int& n_hi) {
+    const long long q0 = (long long)m * kBM;
+    long long lo = p.left >= 0 ? q0 - p.left : 0;
+    long long hi = p.right >= 0 ? q0 + kBM + p.right : len;  // exclusive
+    if (lo < 0) lo = 0;
+    if (hi > len) hi = len;
+    n_lo = (int)(lo / kBN);
+    n_hi = hi > lo ? (int)((hi + kBN - 1) / kBN) : n_lo;
+}
+
+// K-major operand (rows x d, 128-byte swizzle, 64-column boxes 16 KB apart):
+// descriptor of the 16-column step kk.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
+    return ptx::smem_desc_sw128(tile + (kk / 4) * kBoxBytes + (kk % 4) * 32, 16, 1024);
+}
+
+// MN-major B operand ([K rows, N = d columns], N contiguous): the 16-row step kk.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) {
+    return ptx::smem_desc_sw128(tile + kk * 2048, kBoxBytes, 1024);
+}
+
+// ------------------------------------------------------------ D = rowsum(dO * O)
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dsum(const BwdParams p) {
+    const int warp = (blockIdx.x * 256 + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    const int nwarps = gridDim.x * 8;
+    const long long tokens = p.cu_seqlens ? (long long)p.N : (long long)p.B * p.N;
+    const long long rows = tokens * p.Hq;
+    constexpr int kPer = D / 32;  // elements per lane (2 or 4)
+    for (long long r = warp; r < rows; r += nwarps) {
+        const long long t = r / p.Hq;
+        const int h = (int)(r % p.Hq);
+        const uint16_t* op = static_cast<const uint16_t*>(p.o) + r * D + lane * kPer;
+        const uint16_t* dp = static_cast<const uint16_t*>(p.dout) + r * D + lane * kPer;
+        float acc = 0.0f;
+        if (kPer == 4) {
+            const uint2 a = *reinterpret_cast<const uint2*>(op);
+            const uint2 c = *reinterpret_cast<const uint2*>(dp);
+            acc = __uint_as_float(a.x << 16) * __uint_as_float(c.x << 16) +
+                  __uint_as_float(a.x & 0xffff0000u) * __uint_as_float(c.x & 0xffff0000u) +
+                  __uint_as_float(a.y << 16) * __uint_as_float(c.y << 16) +
+                  __uint_as_float(a.y & 0xffff0000u) * __uint_as_float(c.y & 0xffff0000u);
+        } else {
+            const uint32_t a = *reinterpret_cast<const uint32_t*>(op);
+            const uint32_t c = *reinterpret_cast<const uint32_t*>(dp);
+            acc = __uint_as_float(a << 16) * __uint_as_float(c << 16) +
+                  __uint_as_float(a & 0xffff0000u) * __uint_as_float(c & 0xffff0000u);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+            size_t idx;
+            if (p.cu_seqlens) {
+                idx = (size_t)h * p.N + t;
+            } else {
+                const long long b = t / p.N, i = t % p.N;
+                idx = ((size_t)b * p.Hq + h) * p.N + i;
+            }
+            p.dsum[idx] = acc;
+        }
+    }
+}
+
+// ------------------------------------------------------------ dK, dV
+template <int D, int STAGES>
+struct DkvLayout {
+    static constexpr uint32_t kTile = kBN * D * 2;
+    static constexpr uint32_t kK = 0;
+    static constexpr uint32_t kV = kTile;
+    static constexpr uint32_t kRing = 2 * kTile;
+    static constexpr uint32_t kSlot = 2 * kTile + 1024;  // Q, dO, lse2[128], D[128]
+    static constexpr uint32_t kBar = kRing + STAGES * kSlot;
+    // kv_loaded, slot_full[S], slot_empty[S], st_full, p_ready, done
+    static constexpr uint32_t kNumBars = 4 + 2 * STAGES;
+    static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+    static constexpr uint32_t kBytes = kMisc + 16;
+    static constexpr uint32_t kDynamicBytes = kBytes + 1024;
+
+    static __device__ __forceinline__ uint32_t q(uint32_t base, int s) { return base + kRing + s * kSlot; }
+    static __device__ __forceinline__ uint32_t dout(uint32_t base, int s) { return q(base, s) + kTile; }
+    static __device__ __forceinline__ uint32_t stats(uint32_t base, int s) { return q(base, s) + 2 * kTile; }
+    static __device__ __forceinline__ uint32_t bar_kv(uint32_t base) { return base + kBar; }
+    static __device__ __forceinline__ uint32_t bar_full(uint32_t base, int s) { return base + kBar + 8u * (1 + s); }
+    static __device__ __forceinline__ uint32_t bar_empty(uint32_t base, int s) {
+        return base + kBar + 8u * (1 + STAGES + s);
+    }
+    static __device__ __forceinline__ uint32_t bar_st(uint32_t base) { return base + kBar + 8u * (1 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_p(uint32_t base) { return base + kBar + 8u * (2 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (3 + 2 * STAGES); }
+};
+
+// The (query head, query block) steps of a key block, in loop order.
+struct DkvWork {
+    int b, g, n, start, len, m_lo, m_hi, steps;
+};
+
+__device__ __forceinline__ DkvWork dkv_work(const BwdParams& p) {
+    DkvWork w;
+    const int per_n = p.B * p.Hkv;
+    w.n = blockIdx.x / per_n;  // key block 0 (the most query blocks under a causal mask) first
+    const int rem = blockIdx.x % per_n;
+    w.b = rem / p.Hkv;
+    w.g = rem % p.Hkv;
+    const Seq s = seq_of(p, w.b);
+    w.start = s.start;
+    w.len = s.len;
+    if (w.n * kBN >= w.len) {
+        w.steps = 0;
+        w.m_lo = w.m_hi = 0;
+        return w;
+    }
+    query_blocks(p, w.n, w.len, w.m_lo, w.m_hi);
+    w.steps = p.group * (w.m_hi - w.m_lo);
+    return w;
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void dkv_producer(const DkvWork& w, const BwdParams& p, const CUtensorMap* tm_q,
+                                             const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                             const CUtensorMap* tm_do, uint32_t sbase,
+                                             volatile int* abort_flag, uint8_t* smem) {
+    using L = DkvLayout<D, STAGES>;
+    constexpr int kBoxes = D / 64;
+    const int lane = threadIdx.x % 32;
+    const uint64_t pol_kv = ptx::policy_evict_first();
+    const uint64_t pol_q = ptx::policy_evict_last();  // reread by the other key blocks
+    ptx::mbar_arrive_expect_tx_elect(L::bar_kv(sbase), 2 * L::kTile);
+#pragma unroll
+    for (int bx = 0; bx < kBoxes; ++bx) {
+        ptx::tma_load_2d_elect(sbase + L::kK + bx * kBoxBytes, tm_k, L::bar_kv(sbase), w.g * D + bx * 64,
+                               w.start + w.n * kBN, pol_kv);
+        ptx::tma_load_2d_elect(sbase + L::kV + bx * kBoxBytes, tm_v, L::bar_kv(sbase), w.g * D + bx * 64,
+                               w.start + w.n * kBN, pol_kv);
+    }
+    const int nm = w.m_hi - w.m_lo;
+    int issued = 0;
+    for (int t = 0; t < w.steps; ++t) {
+        const int s = t % STAGES;
+        if (!warp_wait(L::bar_empty(sbase, s), ((t / STAGES) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
+        const int h = w.g * p.group + t / nm;
+        const int m = w.m_lo + t % nm;
+        ptx::mbar_arrive_expect_tx_elect(L::bar_full(sbase, s), 2 * L::kTile);
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) {
+            ptx::tma_load_2d_elect(L::q(sbase, s) + bx * kBoxBytes, tm_q, L::bar_full(sbase, s),
+                                   h * D + bx * 64, w.start + m * kBM, pol_q);
+            ptx::tma_load_2d_elect(L::dout(sbase, s) + bx * kBoxBytes, tm_do, L::bar_full(sbase, s),
+                                   h * D + bx * 64, w.start + m * kBM, pol_q);
+        }
+        // lse2 and D of the block's 128 rows (0 past the sequence's end)
+        float* st = reinterpret_cast<float*>(smem + (L::stats(sbase, s) - sbase));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = m * kBM + lane * 4 + e;
+            float l2 = 0.0f, dd = 0.0f;
+            if (i < w.len) {
+                const size_t idx = stat_index(p, w.b, h, w.start, i);
+                l2 = p.lse[idx] * kLog2e;
+                dd = p.dsum[idx];
+            }
+            st[lane * 4 + e] = l2;
+            st[kBM + lane * 4 + e] = dd;
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(L::bar_full(sbase, s));
+        ++issued;
+    }
+    drain_wait(L::bar_kv(sbase), 0, p.wait_limit_ns);
+    const int first = issued > STAGES ? issued - STAGES : 0;
+    for (int i = first; i < issued; ++i)
+        drain_wait(L::bar_full(sbase, i % STAGES), (i / STAGES) & 1, p.wait_limit_ns);
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, uint32_t tmem, uint32_t sbase,
+                                        volatile int* abort_flag) {
+    using L = DkvLayout<D, STAGES>;
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kBN, kBM, false, false);  // M keys, N queries
+    constexpr uint32_t kIdG = ptx::idesc_bf16_f32(kBN, D, false, true);     // M keys, N = d
+    const unsigned long long lim = p.wait_limit_ns;
+    bool ok = warp_wait(L::bar_kv(sbase), 0, abort_flag, lim);
+    ptx::tc_fence_after_sync();
+    for (int t = 0; ok && t < w.steps; ++t) {
+        const int s = t % STAGES;
+        if (!(ok = warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+        const uint32_t qt = L::q(sbase, s), dot = L::dout(sbase, s);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // S^T = K Q^T
+            ptx::mma_ss_elect(tmem, kmajor_desc(sbase + L::kK, kk), kmajor_desc(qt, kk), kIdS, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // dP^T = V dO^T
+            ptx::mma_ss_elect(tmem + 128, kmajor_desc(sbase + L::kV, kk), kmajor_desc(dot, kk), kIdS,
+                              kk > 0 ? 1u : 0u);
+        ptx::tc_commit_elect(L::bar_st(sbase));
+        if (!(ok = warp_wait(L::bar_p(sbase), t & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)  // dV += P^T dO
+            ptx::mma_ts_elect(tmem + 256, tmem + 64 + kk * 8, mnmajor_desc(dot, kk), kIdG,
+                              (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)  // dK += dS^T Q
+            ptx::mma_ts_elect(tmem + 384, tmem + 192 + kk * 8, mnmajor_desc(qt, kk), kIdG,
+                              (t > 0 || kk > 0) ? 1u : 0u);
+        ptx::tc_commit_elect(L::bar_empty(sbase, s));
+    }
+    ptx::tc_commit_elect(L::bar_done(sbase));
+    drain_wait(L::bar_done(sbase), 0, lim);
+}
+
+// One thread = one key row (tensor-memory lane); warpgroup x takes query
+// columns [64x, 64x + 64) of every step.
+template <int D, int STAGES>
+__device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParams& p, uint32_t tmem,
+                                                uint32_t sbase, uint8_t* smem, volatile int* abort_flag) {
+    using L = DkvLayout<D, STAGES>;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int x = warp / 4, wq = warp % 4;
+    const int row = wq * 32 + lane;
+    const int key = w.n * kBN + row;  // within the sequence
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tl = tmem + lane_off;
+    const float sl2 = p.scale_log2;
+    const int nm = w.m_hi - w.m_lo;
+    const unsigned long long lim = p.wait_limit_ns;
+    bool ok = true;
+    for (int t = 0; t < w.steps; ++t) {
+        if (!(ok = warp_wait(L::bar_st(sbase), t & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+        const int s = t % STAGES;
+        const int m = w.m_lo + t % nm;
+        const float* st = reinterpret_cast<const float*>(smem + (L::stats(sbase, s) - sbase));
+        const bool full = block_full(p, m, w.n, w.len);
+        uint32_t pp[32], pd[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int col0 = 64 * x + 32 * c;
+            uint32_t sv[32], dv[32];
+            ptx::tmem_ld32_sync(tl + col0, sv);
+            ptx::tmem_ld32_sync(tl + 128 + col0, dv);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const int ql = col0 + i;
+                const float2 l2 = *reinterpret_cast<const float2*>(st + ql);
+                const float2 dd = *reinterpret_cast<const float2*>(st + kBM + ql);
+                float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2.x));
+                float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2.y));
+                if (!full) {
+                    const int q = m * kBM + ql;
+                    if (!(q < w.len && key < w.len && visible(p, q, key))) p0 = 0.0f;
+                    if (!(q + 1 < w.len && key < w.len && visible(p, q + 1, key))) p1 = 0.0f;
+                }
+                const float d0 = p0 * (__uint_as_float(dv[i]) - dd.x);
+                const float d1 = p1 * (__uint_as_float(dv[i + 1]) - dd.y);
+                pp[c * 16 + i / 2] = ptx::pack_bf16x2(p0, p1);
+                pd[c * 16 + i / 2] = ptx::pack_bf16x2(d0, d1);
+            }
+        }
+        // both warpgroups have read their S^T / dP^T columns before either
+        // overwrites the upper halves with P^T / dS^T
+        ptx::tc_fence_before_sync();
+        elem_sync();
+        ptx::tc_fence_after_sync();
+        ptx::tmem_st32(tl + 64 + 32 * x, pp);
+        ptx::tmem_st32(tl + 192 + 32 * x, pd);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before_sync();
+        ptx::mbar_arrive(L::bar_p(sbase));
+    }
+    if (!ok) return;
+    if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
+    ptx::tc_fence_after_sync();
+    // warpgroup 0 stores dV, warpgroup 1 dK (times the scale)
+    const bool store = key < w.len;
+    const float mul = x ? p.scale : 1.0f;
+    uint8_t* out = static_cast<uint8_t*>(x ? p.dk : p.dv) +
+                   ((size_t)(w.start + (store ? key : 0)) * p.Hkv + w.g) * (size_t)D * 2;
+    const uint32_t src = tl + (x ? 384u : 256u);
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        ptx::tmem_ld32_sync(src + cc * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            pk[i] = ptx::pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+        if (store) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                ptx::st_global_v4(out + cc * 64 + u * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+    }
+}
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                 const BwdParams p) {
+    using L = DkvLayout<D, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = ptx::smem_addr(smem);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const DkvWork w = dkv_work(p);
+    if (w.steps == 0) return;  // uniform over the block
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    if (warp == kWarpProducer && lane == 0) {
+        ptx::mbar_init(L::bar_kv(sbase), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(L::bar_full(sbase, s), 2);  // expect_tx arrival + statistics arrival
+            ptx::mbar_init(L::bar_empty(sbase, s), 1);
+        }
+        ptx::mbar_init(L::bar_st(sbase), 1);
+        ptx::mbar_init(L::bar_p(sbase), kElemThreads);
+        ptx::mbar_init(L::bar_done(sbase), 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_do);
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (warp < 8) {
+        dkv_elementwise<D, STAGES>(w, p, tmem, sbase, smem, abort_flag);
+    } else if (warp == kWarpProducer) {
+        dkv_producer<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, &tm_do, sbase, abort_flag, smem);
+    } else {
+        dkv_mma<D, STAGES>(w, p, tmem, sbase, abort_flag);
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    if (warp == kWarpMma) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------ dQ
+template <int D, int STAGES>
+struct DqLayout {
+    static constexpr uint32_t kTile = kBM * D * 2;
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kDO = kTile;
+    static constexpr uint32_t kRing = 2 * kTile;
+    static constexpr uint32_t kSlot = 2 * kTile;  // K, V
+    static constexpr uint32_t kBar = kRing + STAGES * kSlot;
+    // q_loaded, slot_full[S], slot_empty[S], st_full, ds_ready, done
+    static constexpr uint32_t kNumBars = 4 + 2 * STAGES;
+    static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+    static constexpr uint32_t kBytes = kMisc + 16;
+    static constexpr uint32_t kDynamicBytes = kBytes + 1024;
+
+    static __device__ __forceinline__ uint32_t k(uint32_t base, int s) { return base + kRing + s * kSlot; }
+    static __device__ __forceinline__ uint32_t v(uint32_t base, int s) { return k(base, s) + kTile; }
+    static __device__ __forceinline__ uint32_t bar_q(uint32_t base) { return base + kBar; }
+    static __device__ __forceinline__ uint32_t bar_full(uint32_t base, int s) { return base + kBar + 8u * (1 + s); }
+    static __device__ __forceinline__ uint32_t bar_empty(uint32_t base, int s) {
+        return base + kBar + 8u * (1 + STAGES + s);
+    }
+    static __device__ __forceinline__ uint32_t bar_st(uint32_t base) { return base + kBar + 8u * (1 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_ds(uint32_t base) { return base + kBar + 8u * (2 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (3 + 2 * STAGES); }
+};
+
+struct DqWork {
+    int b, h, g, m, start, len, n_lo, n_hi;
+};
+
+__device__ __forceinline__ DqWork dq_work(const BwdParams& p) {
+    DqWork w;
+    const int per_m = p.B * p.Hq;
+    w.m = p.n_blocks - 1 - blockIdx.x / per_m;  // latest rows (most key blocks, causal) first
+    const int rem = blockIdx.x % per_m;
+    w.b = rem / p.Hq;
+    w.h = rem % p.Hq;
+    w.g = w.h / p.group;
+    const Seq s = seq_of(p, w.b);
+    w.start = s.start;
+    w.len = s.len;
+    if (w.m * kBM >= w.len) {
+        w.n_lo = w.n_hi = 0;
+        return w;
+    }
+    key_blocks(p, w.m, w.len, w.n_lo, w.n_hi);
+    return w;
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void dq_producer(const DqWork& w, const BwdParams& p, const CUtensorMap* tm_q,
+                                            const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                            const CUtensorMap* tm_do, uint32_t sbase, volatile int* abort_flag) {
+    using L = DqLayout<D, STAGES>;
+    constexpr int kBoxes = D / 64;
+    const uint64_t pol_q = ptx::policy_evict_first();
+    const uint64_t pol_kv = ptx::policy_evict_last();
+    ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * L::kTile);
+#pragma unroll
+    for (int bx = 0; bx < kBoxes; ++bx) {
+        ptx::tma_load_2d_elect(sbase + L::kQ + bx * kBoxBytes, tm_q, L::bar_q(sbase), w.h * D + bx * 64,
+                               w.start + w.m * kBM, pol_q);
+        ptx::tma_load_2d_elect(sbase + L::kDO + bx * kBoxBytes, tm_do, L::bar_q(sbase), w.h * D + bx * 64,
+                               w.start + w.m * kBM, pol_q);
+    }
+    int issued = 0;
+    for (int n = w.n_lo; n < w.n_hi; ++n) {
+        const int t = n - w.n_lo, s = t % STAGES;
+        if (!warp_wait(L::bar_empty(sbase, s), ((t / STAGES) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
+        ptx::mbar_arrive_expect_tx_elect(L::bar_full(sbase, s), 2 * L::kTile);
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) {
+            ptx::tma_load_2d_elect(L::k(sbase, s) + bx * kBoxBytes, tm_k, L::bar_full(sbase, s),
+                                   w.g * D + bx * 64, w.start + n * kBN, pol_kv);
+            ptx::tma_load_2d_elect(L::v(sbase, s) + bx * kBoxBytes, tm_v, L::bar_full(sbase, s),
+                                   w.g * D + bx * 64, w.start + n * kBN, pol_kv);
+        }
+        ++issued;
+    }
+    drain_wait(L::bar_q(sbase), 0, p.wait_limit_ns);
+    const int first = issued > STAGES ? issued - STAGES : 0;
+    for (int i = first; i < issued; ++i)
+        drain_wait(L::bar_full(sbase, i % STAGES), (i / STAGES) & 1, p.wait_limit_ns);
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint32_t tmem, uint32_t sbase,
+                                       volatile int* abort_flag) {
+    using L = DqLayout<D, STAGES>;
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kBM, kBN, false, false);
+    constexpr uint32_t kIdG = ptx::idesc_bf16_f32(kBM, D, false, true);
+    const unsigned long long lim = p.wait_limit_ns;
+    bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
+    ptx::tc_fence_after_sync();
+    for (int n = w.n_lo; ok && n < w.n_hi; ++n) {
+        const int t = n - w.n_lo, s = t % STAGES;
+        if (!(ok = warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+        const uint32_t kt = L::k(sbase, s), vt = L::v(sbase, s);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // S = Q K^T
+            ptx::mma_ss_elect(tmem, kmajor_desc(sbase + L::kQ, kk), kmajor_desc(kt, kk), kIdS, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // dP = dO V^T
+            ptx::mma_ss_elect(tmem + 128, kmajor_desc(sbase + L::kDO, kk), kmajor_desc(vt, kk), kIdS,
+                              kk > 0 ? 1u : 0u);
+        ptx::tc_commit_elect(L::bar_st(sbase));
+        if (!(ok = warp_wait(L::bar_ds(sbase), t & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)  // dQ += dS K
+            ptx::mma_ts_elect(tmem + 256, tmem + 64 + kk * 8, mnmajor_desc(kt, kk), kIdG,
+                              (t > 0 || kk > 0) ? 1u : 0u);
+        ptx::tc_commit_elect(L::bar_empty(sbase, s));
+    }
+    ptx::tc_commit_elect(L::bar_done(sbase));
+    drain_wait(L::bar_done(sbase), 0, lim);
+}
+
+// One thread = one query row; warpgroup x takes key columns [64x, 64x + 64).
+template <int D, int STAGES>
+__device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams& p, uint32_t tmem,
+                                               uint32_t sbase, volatile int* abort_flag) {
+    using L = DqLayout<D, STAGES>;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int x = warp / 4, wq = warp % 4;
+    const int row = wq * 32 + lane;
+    const int q = w.m * kBM + row;  // within the sequence
+    const bool valid = q < w.len;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tl = tmem + lane_off;
+    const float sl2 = p.scale_log2;
+    float l2 = 0.0f, dd = 0.0f;
+    if (valid) {
+        const size_t idx = stat_index(p, w.b, w.h, w.start, q);
+        l2 = p.lse[idx] * kLog2e;
+        dd = p.dsum[idx];
+    }
+    const unsigned long long lim = p.wait_limit_ns;
+    bool ok = true;
+    for (int n = w.n_lo; n < w.n_hi; ++n) {
+        const int t = n - w.n_lo;
+        if (!(ok = warp_wait(L::bar_st(sbase), t & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+        const bool full = block_full(p, w.m, n, w.len);
+        uint32_t pd[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int col0 = 64 * x + 32 * c;
+            uint32_t sv[32], dv[32];
+            ptx::tmem_ld32_sync(tl + col0, sv);
+            ptx::tmem_ld32_sync(tl + 128 + col0, dv);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2));
+                float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2));
+                if (!full) {
+                    const int k = n * kBN + col0 + i;
+                    if (!(valid && k < w.len && visible(p, q, k))) p0 = 0.0f;
+                    if (!(valid && k + 1 < w.len && visible(p, q, k + 1))) p1 = 0.0f;
+                }
+                pd[c * 16 + i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd),
+                                                      p1 * (__uint_as_float(dv[i + 1]) - dd));
+            }
+        }
+        ptx::tc_fence_before_sync();
+        elem_sync();
+        ptx::tc_fence_after_sync();
+        ptx::tmem_st32(tl + 64 + 32 * x, pd);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before_sync();
+        ptx::mbar_arrive(L::bar_ds(sbase));
+    }
+    if (!ok) return;
+    if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
+    ptx::tc_fence_after_sync();
+    // warpgroup x stores columns [x * D/2, (x + 1) * D/2) of dQ (times the scale)
+    uint8_t* out = static_cast<uint8_t*>(p.dq) +
+                   ((size_t)(w.start + (valid ? q : 0)) * p.Hq + w.h) * (size_t)D * 2 + x * D;
+#pragma unroll
+    for (int cc = 0; cc < D / 64; ++cc) {
+        uint32_t v[32];
+        ptx::tmem_ld32_sync(tl + 256 + x * (D / 2) + cc * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            pk[i] = ptx::pack_bf16x2(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
+        if (valid) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                ptx::st_global_v4(out + cc * 64 + u * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+    }
+}
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+    using L = DqLayout<D, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = ptx::smem_addr(smem);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const DqWork w = dq_work(p);
+    if (w.n_hi <= w.n_lo) return;  // uniform over the block
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    if (warp == kWarpProducer && lane == 0) {
+        ptx::mbar_init(L::bar_q(sbase), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(L::bar_full(sbase, s), 1);
+            ptx::mbar_init(L::bar_empty(sbase, s), 1);
+        }
+        ptx::mbar_init(L::bar_st(sbase), 1);
+        ptx::mbar_init(L::bar_ds(sbase), kElemThreads);
+        ptx::mbar_init(L::bar_done(sbase), 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_do);
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (warp < 8) {
+        dq_elementwise<D, STAGES>(w, p, tmem, sbase, abort_flag);
+    } else if (warp == kWarpProducer) {
+        dq_producer<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, &tm_do, sbase, abort_flag);
+    } else {
+        dq_mma<D, STAGES>(w, p, tmem, sbase, abort_flag);
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    if (warp == kWarpMma) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace bwd
+}  // namespace attn

@@ -6,4 +6,6 @@ namespace attn {
 // Read and clear the decode kernels' device status word; returns ATTN_OK or
 // ATTN_ERR_CUDA.
 int decode_status_take(int* value);
+// The same for the backward kernels.
+int bwd_status_take(int* value);
 }  // namespace attn

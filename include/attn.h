@@ -110,6 +110,36 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
                   size_t workspace_bytes, struct CUstream_st* stream);
 
 /*
+ * attn_bwd -- gradients of attn_fwd's output with respect to q, k and v
+ * ("FlashAttention" explainer page, How it works, Step 5, and "Backward pass
+ * in a bit more detail": the score tiles are recomputed from q and k and the
+ * weights rebuilt from each row's saved log-sum-exp; key/value gradients
+ * accumulate over query blocks, query gradients over key blocks).
+ *
+ * With P = softmax(scale * q k^T + mask) (from lse), dP = dout v^T,
+ * D = rowsum(dout * o) and dS = P * (dP - D):
+ *     dq = scale * dS k,   dk = scale * dS^T q,   dv = P^T dout,
+ * dk and dv summed over the query heads that share a key/value head.
+ *   q, o, dout, dq [tokens, Hq, d] bf16;  k, v, dk, dv [tokens, Hkv, d] bf16;
+ *   lse: the forward's fp32 log-sum-exp ([B, Hq, N] dense, [Hq, T] packed).
+ *   Sizes, masks, cu_seqlens and max_seqlen as in attn_fwd (same values as the
+ *   forward call that produced o and lse).
+ *   workspace: device, 256-byte aligned, >= attn_bwd_workspace_bytes(...)
+ *   (holds D).  P and dS are rounded to bf16 as operands of the products,
+ *   accumulation is fp32, outputs are rounded once to bf16.
+ * Asynchronous on `stream`; allocates nothing.  Returns ATTN_OK (also for
+ * N == 0, with nothing enqueued) or a negative attn_status; device-side
+ * timeouts are reported by attn_device_status().
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+             float scale, int causal, int window_left, int window_right, const int32_t* cu_seqlens,
+             int max_seqlen, void* workspace, size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Device workspace attn_bwd needs (packed: nonzero when cu_seqlens is passed). */
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int packed);
+
+/*
  * attn_decode -- attention of the newest tokens against a key/value cache,
  * split along the cache ("FlashAttention" explainer page, How it works, Step 9:
  * decoding with a cache of past keys and values; the slices' partial results
