@@ -2,7 +2,7 @@
 """Benchmark of the fused attention forward (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5|decode]
-                    [--impl reference]
+                    [--pass fwd|bwd] [--impl reference]
 
 A step is one call of the fused forward (the whole hot path) over one batch of
 the workload.  The default workload is the causal grouped-query forward at
@@ -23,6 +23,10 @@ collective on the data path.
 
 --impl reference times the CPU oracle (fp64, all host cores) on bounded
 samples of the same workload (rank 0 only).
+
+--pass bwd times attn_bwd (dQ, dK, dV) on the same workload instead, with O and
+LSE from one untimed attn_fwd; the metric counts five products of 2 * d FLOPs
+per visible pair (2.5x the forward's count).
 
 --workload decode times the key/value-cache decode instead (attn_decode: one
 new token for each of 64 sequences against 8192-token paged caches, 32 query
@@ -592,6 +596,239 @@ def run_reference(args, w: W.Workload):
     }
 
 
+# ---------------------------------------------------------------------------
+# backward pass
+# ---------------------------------------------------------------------------
+BWD_METRIC = "attn bwd TFLOP/s (bf16, dQ dK dV, 2.5x the forward's pair count) and % of B200 dense BF16 peak"
+
+
+def bwd_flops_of(w: W.Workload) -> float:
+    """Five products (S, dP, dV, dK, dQ) of 2 * d FLOPs per visible pair: 2.5x the forward."""
+    return 10.0 * w.d * visible_pairs(w) * w.Hq
+
+
+def draw_dout(w: W.Workload, q):
+    import torch
+    g = torch.Generator().manual_seed(w.seed + 1000)
+    return torch.randn(tuple(q.shape), dtype=torch.float32, generator=g).to(torch.bfloat16)
+
+
+def run_bwd(args, w: W.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_142_b200 as ea
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    q, k, v = W.inputs(w)
+    do = draw_dout(w, q)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=dev) if w.packed else None
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.Hq * w.tokens,), dtype=torch.float32, device=dev)
+    ea.attn_fwd(qd, kd, vd, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                w.window_left, w.window_right, cu, w.max_seqlen)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    nbytes = ea.attn_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d, w.packed)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale,
+                    w.causal, w.window_left, w.window_right, cu, w.max_seqlen, ws, nbytes, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported a timeout during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.mark_end()
+    kernel_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported a timeout during the timed region")
+
+    # end to end: the step's inputs (q, k, v, o, lse, dout) copied in from pinned
+    # host memory and the three gradients copied out, every step
+    host_in = [t.cpu().pin_memory() for t in (qd, kd, vd, o, lse, dod)]
+    dev_in = [qd, kd, vd, o, lse, dod]
+    host_out = [torch.empty(tuple(t.shape), dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+
+    def e2e_step():
+        for h, d_ in zip(host_in, dev_in):
+            d_.copy_(h, non_blocking=True)
+        step()
+        for h, d_ in zip(host_out, (dq, dk, dv)):
+            h.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(3, min(args.steps, 20))
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(e_steps):
+        es[i].record(stream)
+        e2e_step()
+        ee[i].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(es, ee)) / e_steps
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([kernel_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        kernel_ms, e2e_ms = float(t[0]), float(t[1])
+    return kernel_ms, e2e_ms, h2d, d2h, clocks
+
+
+def bwd_oracle_sample(w: W.Workload, q, k, v, do, L: int, seed: int):
+    """The oracle's backward on a prefix of L tokens of one sequence and one
+    key/value head group; returns (seconds, algorithmic FLOPs of it, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    lengths = ([b - a for a, b in zip(w.cu_seqlens[:-1], w.cu_seqlens[1:])] if w.packed
+               else [w.N] * w.B)
+    b = int(rng.integers(len(lengths)))
+    while lengths[b] == 0:
+        b = int(rng.integers(len(lengths)))
+    g = int(rng.integers(w.Hkv))
+    L = min(L, lengths[b])
+    grp = w.Hq // w.Hkv
+    start = w.cu_seqlens[b] if w.packed else 0
+
+    def cut(t, heads):
+        if w.packed:
+            x = t[start:start + L, heads]
+        else:
+            x = t[b, :L, heads]
+        return x.unsqueeze(0).contiguous()
+
+    hq = slice(g * grp, (g + 1) * grp)
+    hk = slice(g, g + 1)
+    sub = W.Workload("sample", 1, grp, 1, L, w.d, w.causal, w.window_left, w.window_right, 0)
+    t0 = time.perf_counter()
+    oracle.attn_bwd(W.bf16_bits(cut(q, hq)), W.bf16_bits(cut(k, hk)), W.bf16_bits(cut(v, hk)),
+                    W.bf16_bits(cut(do, hq)), B=1, Hq=grp, Hkv=1, N=L, d=w.d, scale=w.scale,
+                    causal=w.causal, window_left=w.window_left, window_right=w.window_right)
+    return time.perf_counter() - t0, bwd_flops_of(sub), oracle.num_threads()
+
+
+def bwd_calibrate(w, q, k, v, do, target_s):
+    L = 256
+    dt, _, _ = bwd_oracle_sample(w, q, k, v, do, L, seed=1)
+    while dt < 0.5 and L < w.max_seqlen:
+        L *= 2
+        dt, _, _ = bwd_oracle_sample(w, q, k, v, do, L, seed=1)
+    # cost grows with L^2 (causal) or L * window
+    return max(64, min(w.max_seqlen, int(L * math.sqrt(target_s / max(dt, 1e-6)))))
+
+
+def bwd_cpu_baseline(w: W.Workload, target_s: float = 12.0):
+    q, k, v = W.inputs(w)
+    do = draw_dout(w, q)
+    L = bwd_calibrate(w, q, k, v, do, target_s)
+    dt, fl, thr = bwd_oracle_sample(w, q, k, v, do, L, seed=2)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"the first {L} tokens of one sequence, one key/value head group "
+                      f"({w.Hq // w.Hkv} query heads), fp64 oracle backward, {dt:.1f} s "
+                      f"on {thr} threads"}
+
+
+def main_bwd(args, w: W.Workload, rank, world, local_rank):
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        q, k, v = W.inputs(w)
+        do = draw_dout(w, q)
+        budget_s = 150.0 / max(1, args.steps + args.warmup)
+        L = bwd_calibrate(w, q, k, v, do, min(budget_s, 30.0))
+        for i in range(args.warmup):
+            bwd_oracle_sample(w, q, k, v, do, L, seed=10 + i)
+        tot_t, tot_f, thr = 0.0, 0.0, 1
+        for i in range(args.steps):
+            dt, fl, thr = bwd_oracle_sample(w, q, k, v, do, L, seed=1000 + i)
+            tot_t += dt
+            tot_f += fl
+        value = tot_f / tot_t / 1e12
+        print(json.dumps({
+            "metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(config_dict(w, args.gpus), **{"pass": "bwd"}),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": f"a {L}-token prefix of one sequence and head group "
+                                       f"per step; fp64 oracle on {thr} threads"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        kernel_ms, e2e_ms, h2d, d2h, clocks = run_bwd(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.barrier()
+    if rank == 0:
+        fl = bwd_flops_of(w)
+        achieved = fl / (kernel_ms * 1e-3) / 1e12
+        peaks, src = measured_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        line = {
+            "metric": BWD_METRIC, "value": achieved * world, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": kernel_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal bf16 Q, K, V, dO; O and LSE from attn_fwd)",
+            "config": dict(config_dict(w, world), **{"pass": "bwd", "flop_per_step": fl}),
+            "e2e": {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{src} bf16_tflops (burst, cuBLAS)" if src == "measured"
+                         else "fallback 1590 TF/s",
+                         "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
+                         "kernel": f"attn_bwd_dsum<{w.d}> + attn_bwd_dkv<{w.d}> + attn_bwd_dq<{w.d}>",
+                         "timed_as": "whole attn_bwd call (three kernels)"},
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = bwd_cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def config_dict(w: W.Workload, n_gpus: int):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "N": w.N if not w.packed else None, "tokens": w.tokens, "d": w.d,
@@ -611,6 +848,8 @@ def main():
                     help="decode only: cache slices (0 = attn_decode_default_splits)")
     ap.add_argument("--decode-batch", type=int, default=64,
                     help="decode only: sequences (64 is the benchmark; smaller for profiling)")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: attn_fwd (the benchmark); bwd: attn_bwd on the same workload")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -624,6 +863,9 @@ def main():
         main_decode(args, rank, world, local_rank)
         return
     w = W.workload(int(args.workload))
+    if args.pass_ == "bwd":
+        main_bwd(args, w, rank, world, local_rank)
+        return
 
     if args.impl == "reference":
         if rank == 0:
