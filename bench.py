@@ -28,6 +28,11 @@ samples of the same workload (rank 0 only).
 LSE from one untimed attn_fwd; the metric counts five products of 2 * d FLOPs
 per visible pair (2.5x the forward's count).
 
+--workload ring times the context-parallel ring forward: one causal sequence of
+8192 tokens per rank (B=2, Hq=32, Hkv=8, d=128) split in zigzag chunks, K/V
+passed around the ranks with NCCL (weak scaling); on one GPU the ring is one
+rank with two chunks.
+
 --workload decode times the key/value-cache decode instead (attn_decode: one
 new token for each of 64 sequences against 8192-token paged caches, 32 query
 heads over 8 key/value heads, d = 128).  It is bound by HBM, so its metric is
@@ -829,6 +834,140 @@ def main_bwd(args, w: W.Workload, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------
+# context-parallel ring forward
+# ---------------------------------------------------------------------------
+RING_METRIC = "attn ring fwd TFLOP/s (bf16, causal, d=128, sequence split across GPUs)"
+
+
+def ring_workload(world: int) -> W.Workload:
+    """8192 tokens per rank (two zigzag chunks of 4096) of one causal GQA
+    sequence per batch entry: B=2, Hq=32, Hkv=8, d=128, N = 8192 * world."""
+    return W.Workload(f"ring_causal_gqa_b2_hq32_hkv8_n{8192 * world}_d128", 2, 32, 8, 8192 * world,
+                      128, True, -1, -1, 6)
+
+
+def main_ring(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import exact_attention_142_b200 as ea
+    from exact_attention_142_b200 import ring
+
+    w = ring_workload(world)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the ring's reference arm is the oracle forward on the whole "
+                              "sequence; see --workload 3 --impl reference"}), flush=True)
+        return
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    ea.load_library()
+    # this rank's chunks only: draw the rank's slice of a seeded sequence
+    C = w.N // (2 * world)
+    g = torch.Generator(device="cuda").manual_seed(w.seed)
+    full = [torch.randn((w.B, w.N, h, w.d), generator=g, device=dev).to(torch.bfloat16)
+            for h in (w.Hq, w.Hkv, w.Hkv)]
+    qs, ks, vs = (ring.shard_zigzag(t, world, rank) for t in full)
+    del full
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        return ring.ring_attention_forward(qs, ks, vs, scale=w.scale, causal=True,
+                                           group=None, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.mark_end()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported a timeout during the timed region")
+    # end to end: this rank's chunks from pinned host memory, O and LSE back
+    host_in = [t.cpu().pin_memory() for t in (*qs, *ks, *vs)]
+    dev_in = [*qs, *ks, *vs]
+
+    def e2e_step():
+        for h, d_ in zip(host_in, dev_in):
+            d_.copy_(h, non_blocking=True)
+        outs, lses = step()
+        return [x.to("cpu", non_blocking=True) for x in (*outs, *lses)]
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    if world > 1:
+        dist.barrier()
+    for i in range(5):
+        es[i].record(stream)
+        res = e2e_step()
+        ee[i].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(es, ee)) / 5
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in res)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    if rank == 0:
+        fl = flops_of(w)
+        achieved = fl / world / (ms * 1e-3) / 1e12
+        peaks, src = measured_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        pairs = sum(len(pp) for _, _, pp in ring.ring_schedule(world, 0, True))
+        print(json.dumps({
+            "metric": RING_METRIC, "value": fl / (ms * 1e-3) / 1e12, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal bf16 Q, K, V drawn on the device)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N,
+                       "d": w.d, "causal": True, "tokens_per_rank": 2 * C,
+                       "chunk_pairs_per_rank": pairs, "flop_per_step": fl,
+                       "l2": "flushed between timed steps",
+                       "parallelism": f"context parallel x{world} (zigzag ring, NCCL send/recv)"},
+            "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world},
+            "gpu_launches": (pairs + 2) * args.steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{src} bf16_tflops (burst, cuBLAS)" if src == "measured"
+                         else "fallback 1590 TF/s",
+                         "kernel": "attn_fwd_sm100<128,5,accumulate> + attn_acc_to_bf16",
+                         "timed_as": "whole ring step per rank (all chunk pairs, transfers, cast)"},
+            "clocks": clocks,
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def config_dict(w: W.Workload, n_gpus: int):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "N": w.N if not w.packed else None, "tokens": w.tokens, "d": w.d,
@@ -843,7 +982,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="3", choices=["1", "2", "3", "4", "5", "decode"])
+    ap.add_argument("--workload", default="3", choices=["1", "2", "3", "4", "5", "decode", "ring"])
     ap.add_argument("--splits", type=int, default=0,
                     help="decode only: cache slices (0 = attn_decode_default_splits)")
     ap.add_argument("--decode-batch", type=int, default=64,
@@ -861,6 +1000,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.workload == "decode":
         main_decode(args, rank, world, local_rank)
+        return
+    if args.workload == "ring":
+        main_ring(args, rank, world, local_rank)
         return
     w = W.workload(int(args.workload))
     if args.pass_ == "bwd":

@@ -54,6 +54,10 @@ def load_library():
         P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         lib.attn_fwd.restype = I
         lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P]
+        lib.attn_fwd_accumulate.restype = I
+        lib.attn_fwd_accumulate.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P]
+        lib.attn_acc_to_bf16.restype = I
+        lib.attn_acc_to_bf16.argtypes = [P, P, ctypes.c_longlong, P]
         lib.attn_fwd_host.restype = I
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P, S, P]
         lib.attn_fwd_host_workspace_bytes.restype = S
@@ -112,6 +116,27 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window_left
                       int(window_right), _ptr(cu_seqlens), int(max_seqlen), _stream(stream))
     if check and rc != ATTN_OK:
         raise AttnError(rc)
+    return rc
+
+
+def attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, Hq, Hkv, N, d, scale, causal=False,
+                        window_left=-1, window_right=-1, cu_seqlens=None, max_seqlen=0,
+                        stream=None, check=True) -> int:
+    """Merge this call's attention into an fp32 accumulator (see include/attn.h)."""
+    lib = load_library()
+    rc = lib.attn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), int(B),
+                                 int(Hq), int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
+                                 int(window_left), int(window_right), _ptr(cu_seqlens),
+                                 int(max_seqlen), _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_accumulate")
+    return rc
+
+
+def attn_acc_to_bf16(o_acc, o, n, stream=None, check=True) -> int:
+    rc = load_library().attn_acc_to_bf16(_ptr(o_acc), _ptr(o), int(n), _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_acc_to_bf16")
     return rc
 
 

@@ -79,16 +79,20 @@ int prepare_device(int d) {
     }
     if (st.checked < 0) return ATTN_ERR_UNSUPPORTED;
     if (d == 128 && !st.smem_set128) {
-        if (cudaFuncSetAttribute(attn::attn_fwd_sm100<128, kStages128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)attn::SmemLayout<128, kStages128>::kDynamicBytes) != cudaSuccess)
+        const int bytes = (int)attn::SmemLayout<128, kStages128>::kDynamicBytes;
+        if (cudaFuncSetAttribute(attn::attn_fwd_sm100<128, kStages128, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+            cudaFuncSetAttribute(attn::attn_fwd_sm100<128, kStages128, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
             return ATTN_ERR_CUDA;
         st.smem_set128 = true;
     }
     if (d == 64 && !st.smem_set64) {
-        if (cudaFuncSetAttribute(attn::attn_fwd_sm100<64, kStages64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)attn::SmemLayout<64, kStages64>::kDynamicBytes) != cudaSuccess)
+        const int bytes = (int)attn::SmemLayout<64, kStages64>::kDynamicBytes;
+        if (cudaFuncSetAttribute(attn::attn_fwd_sm100<64, kStages64, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+            cudaFuncSetAttribute(attn::attn_fwd_sm100<64, kStages64, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
             return ATTN_ERR_CUDA;
         st.smem_set64 = true;
     }
@@ -119,11 +123,11 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
 }
 
-template <int D, int STAGES>
+template <int D, int STAGES, bool ACC>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
            long long units, cudaStream_t stream) {
-    attn::attn_fwd_sm100<D, STAGES><<<(unsigned)units, attn::kThreads,
-                                       attn::SmemLayout<D, STAGES>::kDynamicBytes, stream>>>(mq, mk, mv, p);
+    attn::attn_fwd_sm100<D, STAGES, ACC><<<(unsigned)units, attn::kThreads,
+                                            attn::SmemLayout<D, STAGES>::kDynamicBytes, stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -131,10 +135,12 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
 
-extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
-                        int window_right, const int32_t* cu_seqlens, int max_seqlen,
-                        struct CUstream_st* stream) {
+namespace {
+
+// The forward pass; acc selects the accumulating epilogue (o is then fp32).
+int run_fwd(bool acc, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+            int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+            int window_right, const int32_t* cu_seqlens, int max_seqlen, cudaStream_t s) {
     const bool packed = cu_seqlens != nullptr;
     long long tokens = 0;
     int rc = validate(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, window_left, window_right, packed,
@@ -173,9 +179,65 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
                                 : (long long)((p.n_row_blocks + 1) / 2) * B * Hq;
     if (units <= 0) return ATTN_OK;
     if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return d == 128 ? launch<128, kStages128>(mq, mk, mv, p, units, s)
-                    : launch<64, kStages64>(mq, mk, mv, p, units, s);
+    if (acc)
+        return d == 128 ? launch<128, kStages128, true>(mq, mk, mv, p, units, s)
+                        : launch<64, kStages64, true>(mq, mk, mv, p, units, s);
+    return d == 128 ? launch<128, kStages128, false>(mq, mk, mv, p, units, s)
+                    : launch<64, kStages64, false>(mq, mk, mv, p, units, s);
+}
+
+}  // namespace
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                        int window_right, const int32_t* cu_seqlens, int max_seqlen,
+                        struct CUstream_st* stream) {
+    return run_fwd(false, q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window_left,
+                   window_right, cu_seqlens, max_seqlen, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc,
+                                   float* lse_acc, int B, int Hq, int Hkv, int N, int d,
+                                   float scale, int causal, int window_left, int window_right,
+                                   const int32_t* cu_seqlens, int max_seqlen,
+                                   struct CUstream_st* stream) {
+    return run_fwd(true, q, k, v, o_acc, lse_acc, B, Hq, Hkv, N, d, scale, causal, window_left,
+                   window_right, cu_seqlens, max_seqlen, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+// fp32 accumulator -> bf16 (round to nearest even), 8 values per thread.
+__global__ void acc_to_bf16_kernel(const float* in, uint16_t* out, long long n) {
+    const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (i + 8 <= n) {
+        const float4 a = *reinterpret_cast<const float4*>(in + i);
+        const float4 b = *reinterpret_cast<const float4*>(in + i + 4);
+        uint4 r;
+        r.x = attn::ptx::pack_bf16x2(a.x, a.y);
+        r.y = attn::ptx::pack_bf16x2(a.z, a.w);
+        r.z = attn::ptx::pack_bf16x2(b.x, b.y);
+        r.w = attn::ptx::pack_bf16x2(b.z, b.w);
+        *reinterpret_cast<uint4*>(out + i) = r;
+    } else {
+        for (long long j = i; j < n; ++j)
+            out[j] = static_cast<uint16_t>(attn::ptx::pack_bf16x2(in[j], 0.0f) & 0xffffu);
+    }
+}
+
+}  // namespace
+
+extern "C" int attn_acc_to_bf16(const float* o_acc, void* o, long long n, struct CUstream_st* stream) {
+    if (n < 0) return ATTN_ERR_SHAPE;
+    if (n == 0) return ATTN_OK;
+    if (!o_acc || !o) return ATTN_ERR_NULL;
+    if (!aligned(o_acc, 16) || !aligned(o, 16)) return ATTN_ERR_ALIGN;
+    const long long threads = (n + 7) / 8;
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+    acc_to_bf16_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        o_acc, static_cast<uint16_t*>(o), n);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 extern "C" size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int packed) {

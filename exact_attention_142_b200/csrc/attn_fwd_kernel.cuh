@@ -57,6 +57,7 @@ constexpr uint32_t kTmemO0 = 256;
 constexpr uint32_t kPOffset = 64;      // P columns inside an S region
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kLog2e = 1.442695040888963407f;
 // Register split after launch (384 threads x 168 = 64512 registers):
 // 128 x (216 + 216 + 72) = 64512.
 constexpr uint32_t kRegsSoftmax = 216;
@@ -403,7 +404,11 @@ __device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, 
 }
 
 // ---------------------------------------------------------------- softmax
-template <int D, int STAGES>
+// ACC = false: O (bf16) and LSE are written.  ACC = true: this call's result is
+// merged into an fp32 accumulator (o as float [tokens, Hq, d], lse holding the
+// accumulator's log-sum-exp) by the online-softmax rule (Step 3 applied to two
+// partial results; "Long context beyond a single GPU").
+template <int D, int STAGES, bool ACC>
 __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams& p, int x,
                                              int warp_in_group, int lane, uint32_t tmem,
                                              uint32_t sbase, volatile int* abort_flag) {
@@ -551,6 +556,41 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
     if (!ok) return;
     ptx::tc_fence_after_sync();
     const bool store = row < w.len;
+    if constexpr (ACC) {
+        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + w.start + (store ? row : 0)
+                                        : ((size_t)w.b * p.Hq + h) * p.N + (store ? row : 0);
+        // both log-sum-exps in log2 units; weights relative to the larger one
+        const float lse_new = l_sum > 0.0f ? m_ref + ptx::lg2_approx(l_sum) : -INFINITY;
+        const float lse_old = store ? p.lse[idx] * kLog2e : -INFINITY;
+        const float mx = fmaxf(lse_old, lse_new);
+        const float mu = mx == -INFINITY ? 0.0f : mx;
+        const float w_old = ptx::ex2_approx(lse_old - mu);
+        const float w_new = ptx::ex2_approx(lse_new - mu);
+        const float den = w_old + w_new;
+        const float inv_den = den > 0.0f ? 1.0f / den : 0.0f;
+        const float a_old = w_old * inv_den;
+        const float a_new = l_bf > 0.0f ? w_new * inv_den / l_bf : 0.0f;
+        float* acc = static_cast<float*>(p.o) + ((size_t)(w.start + (store ? row : 0)) * p.Hq + h) * (size_t)D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            ptx::tmem_ld32_sync(t_o + cc * 32, o);
+            if (store) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    float4* ap = reinterpret_cast<float4*>(acc + cc * 32 + v * 4);
+                    float4 a = *ap;
+                    a.x = fmaf(a_old, a.x, a_new * __uint_as_float(o[4 * v + 0]));
+                    a.y = fmaf(a_old, a.y, a_new * __uint_as_float(o[4 * v + 1]));
+                    a.z = fmaf(a_old, a.z, a_new * __uint_as_float(o[4 * v + 2]));
+                    a.w = fmaf(a_old, a.w, a_new * __uint_as_float(o[4 * v + 3]));
+                    *ap = a;
+                }
+            }
+        }
+        if (store) p.lse[idx] = den > 0.0f ? (mu + ptx::lg2_approx(den)) * kLn2 : -INFINITY;
+        return;
+    }
     const float inv = l_bf > 0.0f ? 1.0f / l_bf : 0.0f;
     uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
                     ((size_t)(w.start + (store ? row : 0)) * p.Hq + h) * (size_t)D * 2;
@@ -578,7 +618,7 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, int STAGES>
+template <int D, int STAGES, bool ACC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -625,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
-        softmax_role<D, STAGES>(w, p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
+        softmax_role<D, STAGES, ACC>(w, p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (warp == kWarpProducer) {

@@ -88,6 +88,31 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              const int32_t* cu_seqlens, int max_seqlen, struct CUstream_st* stream);
 
 /*
+ * attn_fwd_accumulate -- attn_fwd whose result is merged into an fp32
+ * accumulator instead of being written: the building block of attention split
+ * along the keys ("Long context beyond a single GPU": devices compute partial
+ * attention and merge the partial results with the online-softmax rule of
+ * "How it works", Step 3).
+ *   o_acc   [tokens, Hq, d] fp32 and lse_acc (laid out like lse) hold a
+ *           partial result over some other keys; a row whose lse_acc is -inf
+ *           holds nothing yet (start from o_acc = 0, lse_acc = -inf).
+ * With (O', L') this call's attention of q over k, v (natural-log LSE), each
+ * row becomes  L = log(e^lse_acc + e^L'),
+ *              o_acc = (e^lse_acc o_acc + e^L' O') / e^L,   lse_acc = L,
+ * so that after all key blocks o_acc and lse_acc are attn_fwd's O (before
+ * rounding) and LSE for all the keys.  Every other argument, rule and status is
+ * attn_fwd's; o_acc must be 16-byte aligned.
+ */
+int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc,
+                        int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                        int window_left, int window_right, const int32_t* cu_seqlens,
+                        int max_seqlen, struct CUstream_st* stream);
+
+/* Round n fp32 values (an accumulator) to bf16, nearest even; both buffers
+ * 16-byte aligned device memory.  Asynchronous on `stream`. */
+int attn_acc_to_bf16(const float* o_acc, void* o, long long n, struct CUstream_st* stream);
+
+/*
  * attn_fwd_host_workspace_bytes -- device workspace needed by attn_fwd_host
  * for these sizes (q, k, v, o, lse and cu_seqlens copies, 256-byte aligned).
  * packed: nonzero when cu_seqlens will be passed.  Returns 0 on bad sizes.
