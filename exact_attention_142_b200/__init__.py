@@ -11,7 +11,8 @@ from ._binding import (  # noqa: F401
     ATTN_DECODE_NOALLOC_SCRATCH_BYTES, attn_bwd, attn_bwd_workspace_bytes, attn_decode,
     attn_decode_default_splits,
     attn_decode_noalloc, attn_decode_workspace_bytes, attn_device_status,
-    attn_acc_to_bf16, attn_fwd, attn_fwd_accumulate, attn_fwd_host, attn_fwd_host_workspace_bytes,
+    attn_acc_to_bf16, attn_fwd, attn_fwd_accumulate, attn_fwd_fp8, attn_fwd_fp8_workspace_bytes,
+    attn_fwd_host, attn_fwd_host_workspace_bytes,
     attn_selftest_bounded_wait, attn_status_string, library_path, load_library)
 
 

@@ -54,6 +54,10 @@ def load_library():
         P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         lib.attn_fwd.restype = I
         lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P]
+        lib.attn_fwd_fp8.restype = I
+        lib.attn_fwd_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P, S, P]
+        lib.attn_fwd_fp8_workspace_bytes.restype = S
+        lib.attn_fwd_fp8_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.attn_fwd_accumulate.restype = I
         lib.attn_fwd_accumulate.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I, P]
         lib.attn_acc_to_bf16.restype = I
@@ -117,6 +121,25 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window_left
     if check and rc != ATTN_OK:
         raise AttnError(rc)
     return rc
+
+
+def attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal=False, window_left=-1,
+                 window_right=-1, cu_seqlens=None, max_seqlen=0, workspace=None, workspace_bytes=0,
+                 stream=None, check=True) -> int:
+    """The fused forward on e4m3 inputs (see include/attn.h)."""
+    lib = load_library()
+    rc = lib.attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq), int(Hkv),
+                          int(N), int(d), float(scale), int(bool(causal)), int(window_left),
+                          int(window_right), _ptr(cu_seqlens), int(max_seqlen), _ptr(workspace),
+                          int(workspace_bytes), _stream(stream))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_fp8")
+    return rc
+
+
+def attn_fwd_fp8_workspace_bytes(B, Hq, Hkv, N, d, packed) -> int:
+    return int(load_library().attn_fwd_fp8_workspace_bytes(int(B), int(Hq), int(Hkv), int(N), int(d),
+                                                           int(bool(packed))))
 
 
 def attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, Hq, Hkv, N, d, scale, causal=False,

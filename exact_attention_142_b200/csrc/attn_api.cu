@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "attn_fwd_fp8_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 #include "attn_internal.h"
 
@@ -54,10 +55,24 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, cols] one-byte elements in boxes of 128 rows x 128 bytes, 128-byte
+// swizzle (the e4m3 tiles); rows past the end read as zero.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estride[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr int kMaxDevices = 64;
 struct DeviceState {
     int checked = 0;  // 1 = supported, -1 = unsupported
-    bool smem_set64 = false, smem_set128 = false;
+    bool smem_set64 = false, smem_set128 = false, smem_set_fp8 = false;
 };
 DeviceState g_devices[kMaxDevices];
 std::mutex g_dev_mu;
@@ -86,6 +101,12 @@ int prepare_device(int d) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
             return ATTN_ERR_CUDA;
         st.smem_set128 = true;
+    }
+    if (d == 8 && !st.smem_set_fp8) {  // d == 8: the e4m3 kernel
+        if (cudaFuncSetAttribute(attn::fp8::attn_fwd_fp8_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)attn::fp8::Layout::kDynamicBytes) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        st.smem_set_fp8 = true;
     }
     if (d == 64 && !st.smem_set64) {
         const int bytes = (int)attn::SmemLayout<64, kStages64>::kDynamicBytes;
@@ -237,6 +258,80 @@ extern "C" int attn_acc_to_bf16(const float* o_acc, void* o, long long n, struct
     if (blocks > 0x7fffffffLL) return ATTN_ERR_SHAPE;
     acc_to_bf16_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         o_acc, static_cast<uint16_t*>(o), n);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- e4m3 inputs
+namespace {
+
+// Columns of the padded V^T: every sequence rounded up to 128 keys fits in
+// tokens + 128 * B; rounded to 16 bytes for the tensor map's row stride.
+long long vt_columns(int B, long long tokens) { return (tokens + 128LL * B + 15) / 16 * 16; }
+
+}  // namespace
+
+extern "C" size_t attn_fwd_fp8_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int packed) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d != 128 || Hq % Hkv) return 0;
+    const long long tokens = packed ? (long long)N : (long long)B * N;
+    return round256((size_t)Hkv * 128 * (size_t)vt_columns(B, tokens));
+}
+
+extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                            int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                            int window_right, const int32_t* cu_seqlens, int max_seqlen,
+                            void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
+    const bool packed = cu_seqlens != nullptr;
+    long long tokens = 0;
+    int rc = validate(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, window_left, window_right, packed,
+                      max_seqlen, &tokens);
+    if (rc != ATTN_OK) return rc;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (tokens == 0) return ATTN_OK;
+    if (B > 65535) return ATTN_ERR_SHAPE;
+    const size_t need = attn_fwd_fp8_workspace_bytes(B, Hq, Hkv, N, d, packed ? 1 : 0);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
+    rc = prepare_device(8);
+    if (rc != ATTN_OK) return rc;
+    const long long vt_cols = vt_columns(B, tokens);
+    if (vt_cols > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+
+    CUtensorMap mq, mk, mvt;
+    if (!make_map_u8(&mq, q, (uint64_t)tokens, (uint64_t)Hq * 128) ||
+        !make_map_u8(&mk, k, (uint64_t)tokens, (uint64_t)Hkv * 128) ||
+        !make_map_u8(&mvt, workspace, (uint64_t)Hkv * 128, (uint64_t)vt_cols))
+        return ATTN_ERR_CUDA;
+
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens = cu_seqlens;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.group = Hq / Hkv;
+    p.left = window_left;
+    p.right = causal ? 0 : window_right;
+    p.pair_mode = (p.group % 2 == 0) ? attn::kPairHeads : attn::kPairRows;
+    const int max_len = packed ? (max_seqlen < N ? max_seqlen : N) : N;
+    p.n_row_blocks = (max_len + attn::kBM - 1) / attn::kBM;
+    p.scale = scale;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+    p.wait_limit_ns = kWaitLimitNs;
+    const long long units = p.pair_mode == attn::kPairHeads
+                                ? (long long)p.n_row_blocks * B * (Hq / 2)
+                                : (long long)((p.n_row_blocks + 1) / 2) * B * Hq;
+    if (units <= 0) return ATTN_OK;
+    if (units > 0x7fffffffLL || Hkv > 65535) return ATTN_ERR_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // 64-key blocks up to the longest sequence's padded length (pad columns are zeroed)
+    const dim3 tgrid((unsigned)((max_len + attn::kBN - 1) / attn::kBN * (attn::kBN / 64)), (unsigned)Hkv,
+                     (unsigned)B);
+    attn::fp8::attn_vt_transpose_kernel<<<tgrid, 256, 0, s>>>(static_cast<const uint8_t*>(v),
+                                                               static_cast<uint8_t*>(workspace), p, vt_cols);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    attn::fp8::attn_fwd_fp8_sm100<<<(unsigned)units, attn::kThreads, attn::fp8::Layout::kDynamicBytes, s>>>(
+        mq, mk, mvt, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -88,6 +88,31 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              const int32_t* cu_seqlens, int max_seqlen, struct CUstream_st* stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd with 8-bit floating-point inputs ("Flash Attention"
+ * skill page, Workflow 3: q, k, v converted to float8_e4m3 and passed to the
+ * fused kernel; "FlashAttention" explainer page, How it works, Step 8:
+ * 8-bit products with fp32 statistics).
+ *   q [tokens, Hq, 128], k and v [tokens, Hkv, 128]: e4m3 (OCP "E4M3FN": one
+ *   sign, four exponent, three mantissa bits, bias 7, no infinities), one byte
+ *   each, 16-byte aligned; the values themselves, with no scale factors.
+ *   o bf16 and lse fp32 as in attn_fwd; every other argument as in attn_fwd.
+ *   d must be 128 (ATTN_ERR_UNSUPPORTED otherwise).
+ * Both products take e4m3 operands with fp32 accumulation: the weights P are
+ * rounded to e4m3 (round to nearest even) for O += P V and O is divided by the
+ * sum of those rounded weights; the LSE uses the fp32 weights.
+ * workspace: device, 256-byte aligned, >= attn_fwd_fp8_workspace_bytes(...):
+ * holds V transposed per key/value head, each sequence padded to 128 keys.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int N, int d, float scale, int causal, int window_left, int window_right,
+                 const int32_t* cu_seqlens, int max_seqlen, void* workspace, size_t workspace_bytes,
+                 struct CUstream_st* stream);
+
+/* Device workspace attn_fwd_fp8 needs (packed: nonzero when cu_seqlens is passed;
+ * 0 for d != 128 or bad sizes). */
+size_t attn_fwd_fp8_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int packed);
+
+/*
  * attn_fwd_accumulate -- attn_fwd whose result is merged into an fp32
  * accumulator instead of being written: the building block of attention split
  * along the keys ("Long context beyond a single GPU": devices compute partial

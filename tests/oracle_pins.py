@@ -644,6 +644,35 @@ def pin_bwd_packed_and_grouped(lib):
     assert np.abs(dv - dv2.reshape(T, Hkv, g, d).sum(axis=2)).max() <= 1e-12
 
 
+# --------------------------------------------------------------------------
+# e4m3 inputs
+# --------------------------------------------------------------------------
+def _e4m3_value(code: int) -> float:
+    """E4M3FN from its definition: sign, 4 exponent bits (bias 7), 3 mantissa
+    bits; exponent 0 is subnormal (2^-6 * m/8); S.1111.111 is NaN (no inf)."""
+    s = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        return s * (m / 8.0) * 2.0 ** -6
+    return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def pin_e4m3_widening(lib):
+    """The e4m3 -> bf16 widening that feeds the oracle is exact for all 256
+    codes (checked against the format's definition)."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    widened = W.e4m3_as_bf16(codes.view(torch.float8_e4m3fn)).to(torch.float64).numpy()
+    for c in range(256):
+        want = _e4m3_value(c)
+        if math.isnan(want):
+            assert math.isnan(widened[c])
+        else:
+            assert widened[c] == want, (c, widened[c], want)
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_uniform_scores,
@@ -666,4 +695,5 @@ ALL_PINS = [
     pin_bwd_torch_autograd,
     pin_bwd_invariants,
     pin_bwd_packed_and_grouped,
+    pin_e4m3_widening,
 ]

@@ -200,3 +200,23 @@ def decode_inputs(w: DecodeWorkload, device: str = "cpu"):
         perm = torch.randperm(pages, generator=torch.Generator().manual_seed(w.seed))
         table = perm.to(torch.int32).reshape(w.B, w.pages_per_seq)
     return q, kc, vc, seqlens, table
+
+
+# --------------------------------------------------------------------------
+# 8-bit (e4m3) inputs
+# --------------------------------------------------------------------------
+def draw_qkv_e4m3(shape_q, shape_kv, seed: int):
+    """q, k, v as CPU float8_e4m3fn tensors: the same normal draws as draw_qkv,
+    converted to e4m3 (round to nearest even, as torch's .to(float8_e4m3fn))."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn(shape_q, dtype=torch.float32, generator=g).to(torch.float8_e4m3fn)
+    k = torch.randn(shape_kv, dtype=torch.float32, generator=g).to(torch.float8_e4m3fn)
+    v = torch.randn(shape_kv, dtype=torch.float32, generator=g).to(torch.float8_e4m3fn)
+    return q, k, v
+
+
+def e4m3_as_bf16(t: torch.Tensor) -> torch.Tensor:
+    """Every finite e4m3 value is exact in bf16 (3 mantissa bits into 7, exponents
+    2^-9 .. 2^8 inside bf16's range): the oracle's bf16 input for e4m3 data."""
+    return t.to(torch.bfloat16)
