@@ -2,7 +2,7 @@
 """Benchmark of the fused attention forward (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5|decode]
-                    [--pass fwd|bwd] [--impl reference]
+                    [--pass fwd|bwd] [--dtype bf16|fp8] [--impl reference]
 
 A step is one call of the fused forward (the whole hot path) over one batch of
 the workload.  The default workload is the causal grouped-query forward at
@@ -27,6 +27,9 @@ samples of the same workload (rank 0 only).
 --pass bwd times attn_bwd (dQ, dK, dV) on the same workload instead, with O and
 LSE from one untimed attn_fwd; the metric counts five products of 2 * d FLOPs
 per visible pair (2.5x the forward's count).
+
+--dtype fp8 times attn_fwd_fp8 (e4m3 inputs) on the same workload, against
+the measured bf16 peak x 2 (the nominal fp8 / bf16 tensor-core ratio).
 
 --workload ring times the context-parallel ring forward: one causal sequence of
 8192 tokens per rank (B=2, Hq=32, Hkv=8, d=128) split in zigzag chunks, K/V
@@ -968,6 +971,129 @@ def main_ring(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------
+# e4m3 inputs
+# ---------------------------------------------------------------------------
+FP8_METRIC = "attn fwd TFLOP/s (e4m3 inputs, causal, d=128) and % of B200 dense FP8 peak"
+
+
+def main_fp8(args, w: W.Workload, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import exact_attention_142_b200 as ea
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the e4m3 path's reference arm is the oracle on the widened "
+                              "values; see --impl reference for the bf16 workload"}), flush=True)
+        return
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    ea.load_library()
+    if w.packed:
+        q, k, v = W.draw_qkv_e4m3((w.tokens, w.Hq, w.d), (w.tokens, w.Hkv, w.d), w.seed)
+    else:
+        q, k, v = W.draw_qkv_e4m3((w.B, w.N, w.Hq, w.d), (w.B, w.N, w.Hkv, w.d), w.seed)
+    qd, kd, vd = (t.view(torch.uint8).to(dev) for t in (q, k, v))
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=dev) if w.packed else None
+    o = torch.empty(tuple(q.shape), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.Hq * w.tokens,), dtype=torch.float32, device=dev)
+    nbytes = ea.attn_fwd_fp8_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d, w.packed)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ea.attn_fwd_fp8(qd, kd, vd, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                        w.window_left, w.window_right, cu, w.max_seqlen, ws, nbytes, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.mark_end()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported a timeout during the timed region")
+    host_in = [t.view(torch.uint8).pin_memory() for t in (q, k, v)]
+    oh = torch.empty(tuple(o.shape), dtype=o.dtype).pin_memory()
+    lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for h, d_ in zip(host_in, (qd, kd, vd)):
+            d_.copy_(h, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+    if world > 1:
+        dist.barrier()
+    for i in range(10):
+        es[i].record(stream)
+        e2e_step()
+        ee[i].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(es, ee)) / 10
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    if rank == 0:
+        fl = flops_of(w)
+        achieved = fl / (ms * 1e-3) / 1e12
+        peaks, src = measured_peaks()
+        peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        print(json.dumps({
+            "metric": FP8_METRIC, "value": achieved * world, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic (seeded normal draws rounded to e4m3)",
+            "config": dict(config_dict(w, world), **{"inputs": "e4m3"}),
+            "e2e": {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": sum(t.numel() for t in host_in),
+                    "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4},
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": (f"{src} bf16_tflops x 2 (nominal fp8 / bf16 ratio)"
+                                         if src == "measured" else "fallback 1590 x 2"),
+                         "frac_of_bf16_peak": achieved / (peak / 2),
+                         "kernel": "attn_vt_transpose_kernel + attn_fwd_fp8_sm100",
+                         "timed_as": "whole attn_fwd_fp8 call (transpose + kernel)"},
+            "clocks": clocks,
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def config_dict(w: W.Workload, n_gpus: int):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "N": w.N if not w.packed else None, "tokens": w.tokens, "d": w.d,
@@ -989,6 +1115,8 @@ def main():
                     help="decode only: sequences (64 is the benchmark; smaller for profiling)")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
                     help="fwd: attn_fwd (the benchmark); bwd: attn_bwd on the same workload")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: the forward on e4m3 inputs (attn_fwd_fp8); d = 128 workloads")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -1007,6 +1135,9 @@ def main():
     w = W.workload(int(args.workload))
     if args.pass_ == "bwd":
         main_bwd(args, w, rank, world, local_rank)
+        return
+    if args.dtype == "fp8":
+        main_fp8(args, w, rank, world, local_rank)
         return
 
     if args.impl == "reference":
