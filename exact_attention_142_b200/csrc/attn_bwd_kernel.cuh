@@ -13,7 +13,7 @@
 //                    head of the group and every query block that sees the keys
 //                    stream through a 2-stage ring.  Per query block:
 //                      S^T = K Q^T, dP^T = V dO^T      (tcgen05, both from smem)
-//                      P^T, dS^T                        (8 warps, fp32 -> bf16)
+//                      P^T, dS^T                        (16 warps, fp32 -> bf16)
 //                      dV += P^T dO, dK += dS^T Q       (A from tensor memory)
 //                    dK and dV stay in tensor memory for the whole loop, so each
 //                    key row is written once, already summed over the group.
@@ -24,11 +24,12 @@
 // Tensor memory (512 columns): dkv: S^T [0,128), dP^T [128,256), dV [256,256+d),
 // dK [384,384+d); dq: S [0,128), dP [128,256), dQ [256,256+d).  The bf16 P^T /
 // dS^T (dS) are written into the upper 64 columns of their fp32 source region
-// once both warpgroups have read it, and the next product reads them there.
+// once every column group has read it, and the next product reads them there.
 //
-// Warps: 0-7 elementwise (warpgroup x = warp / 4 takes the tile's columns
-// [64x, 64x + 64); warp w % 4 its 32 tensor-memory lanes), 8 TMA producer,
-// 9 MMA issuer (both converged, one elected lane issues).
+// Warps: 0-15 elementwise (column group x = warp / 4 takes the tile's columns
+// [32x, 32x + 32); warp w % 4 its 32 tensor-memory lanes: four warps per
+// sub-partition hide the latency of the exponentials), 16 TMA producer, 17 MMA
+// issuer (both converged, one elected lane issues).
 #pragma once
 
 #include <cstdint>
@@ -45,10 +46,13 @@ __device__ int g_bwd_status;
 
 constexpr int kBM = 128;  // query rows per block
 constexpr int kBN = 128;  // keys per block
-constexpr int kThreads = 320;
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
-constexpr int kElemThreads = 256;
+constexpr int kElemWarps = 16;              // 4 column groups x 4 lane quadrants
+constexpr int kGroups = kElemWarps / 4;      // column groups
+constexpr int kGroupCols = 128 / kGroups;    // columns of a step per group
+constexpr int kWarpProducer = kElemWarps;
+constexpr int kWarpMma = kElemWarps + 1;
+constexpr int kThreads = (kElemWarps + 2) * 32;
+constexpr int kElemThreads = kElemWarps * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBoxBytes = 128 * 128;  // one TMA box: 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
@@ -103,6 +107,19 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, unsign
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned long long limit_ns) {
     return __all_sync(0xffffffffu, bounded_wait(bar, parity, abort_flag, limit_ns));
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns per thread, then wait.
+__device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
 }
 
 __device__ __forceinline__ void elem_sync() {
@@ -368,8 +385,8 @@ __device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, ui
     drain_wait(L::bar_done(sbase), 0, lim);
 }
 
-// One thread = one key row (tensor-memory lane); warpgroup x takes query
-// columns [64x, 64x + 64) of every step.
+// One thread = one key row (tensor-memory lane); column group x = warp / 4
+// takes query columns [32x, 32x + 32) of every step.
 template <int D, int STAGES>
 __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParams& p, uint32_t tmem,
                                                 uint32_t sbase, uint8_t* smem, volatile int* abort_flag) {
@@ -391,15 +408,15 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
         const int m = w.m_lo + t % nm;
         const float* st = reinterpret_cast<const float*>(smem + (L::stats(sbase, s) - sbase));
         const bool full = block_full(p, m, w.n, w.len);
-        uint32_t pp[32], pd[32];
+        uint32_t pp[kGroupCols / 2], pd[kGroupCols / 2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const int col0 = 64 * x + 32 * c;
-            uint32_t sv[32], dv[32];
-            ptx::tmem_ld32_sync(tl + col0, sv);
-            ptx::tmem_ld32_sync(tl + 128 + col0, dv);
+        for (int c = 0; c < kGroupCols / 16; ++c) {
+            const int col0 = kGroupCols * x + 16 * c;
+            uint32_t sv[16], dv[16];
+            tmem_ld16_sync(tl + col0, sv);
+            tmem_ld16_sync(tl + 128 + col0, dv);
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
+            for (int i = 0; i < 16; i += 2) {
                 const int ql = col0 + i;
                 const float2 l2 = *reinterpret_cast<const float2*>(st + ql);
                 const float2 dd = *reinterpret_cast<const float2*>(st + kBM + ql);
@@ -412,17 +429,17 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
                 }
                 const float d0 = p0 * (__uint_as_float(dv[i]) - dd.x);
                 const float d1 = p1 * (__uint_as_float(dv[i + 1]) - dd.y);
-                pp[c * 16 + i / 2] = ptx::pack_bf16x2(p0, p1);
-                pd[c * 16 + i / 2] = ptx::pack_bf16x2(d0, d1);
+                pp[c * 8 + i / 2] = ptx::pack_bf16x2(p0, p1);
+                pd[c * 8 + i / 2] = ptx::pack_bf16x2(d0, d1);
             }
         }
-        // both warpgroups have read their S^T / dP^T columns before either
-        // overwrites the upper halves with P^T / dS^T
+        // every group has read its S^T / dP^T columns before any overwrites the
+        // upper halves with P^T / dS^T
         ptx::tc_fence_before_sync();
         elem_sync();
         ptx::tc_fence_after_sync();
-        ptx::tmem_st32(tl + 64 + 32 * x, pp);
-        ptx::tmem_st32(tl + 192 + 32 * x, pd);
+        ptx::tmem_st16(tl + 64 + (kGroupCols / 2) * x, pp);
+        ptx::tmem_st16(tl + 192 + (kGroupCols / 2) * x, pd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_p(sbase));
@@ -430,14 +447,16 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
     ptx::tc_fence_after_sync();
-    // warpgroup 0 stores dV, warpgroup 1 dK (times the scale)
+    // groups 0, 1 store the two halves of dV's columns, groups 2, 3 of dK's (times the scale)
     const bool store = key < w.len;
-    const float mul = x ? p.scale : 1.0f;
-    uint8_t* out = static_cast<uint8_t*>(x ? p.dk : p.dv) +
-                   ((size_t)(w.start + (store ? key : 0)) * p.Hkv + w.g) * (size_t)D * 2;
-    const uint32_t src = tl + (x ? 384u : 256u);
+    const bool is_k = x >= 2;
+    const int half = x & 1;
+    const float mul = is_k ? p.scale : 1.0f;
+    uint8_t* out = static_cast<uint8_t*>(is_k ? p.dk : p.dv) +
+                   ((size_t)(w.start + (store ? key : 0)) * p.Hkv + w.g) * (size_t)D * 2 + half * D;
+    const uint32_t src = tl + (is_k ? 384u : 256u) + half * (D / 2);
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
+    for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t v[32];
         ptx::tmem_ld32_sync(src + cc * 32, v);
         uint32_t pk[16];
@@ -491,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    if (warp < 8) {
+    if (warp < kElemWarps) {
         dkv_elementwise<D, STAGES>(w, p, tmem, sbase, smem, abort_flag);
     } else if (warp == kWarpProducer) {
         dkv_producer<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, &tm_do, sbase, abort_flag, smem);
@@ -624,7 +643,8 @@ __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint
     drain_wait(L::bar_done(sbase), 0, lim);
 }
 
-// One thread = one query row; warpgroup x takes key columns [64x, 64x + 64).
+// One thread = one query row; column group x = warp / 4 takes key columns
+// [32x, 32x + 32).
 template <int D, int STAGES>
 __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams& p, uint32_t tmem,
                                                uint32_t sbase, volatile int* abort_flag) {
@@ -650,15 +670,15 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
         if (!(ok = warp_wait(L::bar_st(sbase), t & 1, abort_flag, lim))) break;
         ptx::tc_fence_after_sync();
         const bool full = block_full(p, w.m, n, w.len);
-        uint32_t pd[32];
+        uint32_t pd[kGroupCols / 2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const int col0 = 64 * x + 32 * c;
-            uint32_t sv[32], dv[32];
-            ptx::tmem_ld32_sync(tl + col0, sv);
-            ptx::tmem_ld32_sync(tl + 128 + col0, dv);
+        for (int c = 0; c < kGroupCols / 16; ++c) {
+            const int col0 = kGroupCols * x + 16 * c;
+            uint32_t sv[16], dv[16];
+            tmem_ld16_sync(tl + col0, sv);
+            tmem_ld16_sync(tl + 128 + col0, dv);
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
+            for (int i = 0; i < 16; i += 2) {
                 float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2));
                 float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2));
                 if (!full) {
@@ -666,14 +686,14 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
                     if (!(valid && k < w.len && visible(p, q, k))) p0 = 0.0f;
                     if (!(valid && k + 1 < w.len && visible(p, q, k + 1))) p1 = 0.0f;
                 }
-                pd[c * 16 + i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd),
-                                                      p1 * (__uint_as_float(dv[i + 1]) - dd));
+                pd[c * 8 + i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd),
+                                                     p1 * (__uint_as_float(dv[i + 1]) - dd));
             }
         }
         ptx::tc_fence_before_sync();
         elem_sync();
         ptx::tc_fence_after_sync();
-        ptx::tmem_st32(tl + 64 + 32 * x, pd);
+        ptx::tmem_st16(tl + 64 + (kGroupCols / 2) * x, pd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_ds(sbase));
@@ -681,22 +701,24 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
     ptx::tc_fence_after_sync();
-    // warpgroup x stores columns [x * D/2, (x + 1) * D/2) of dQ (times the scale)
+    // group x stores columns [x * D/4, (x + 1) * D/4) of dQ (times the scale)
+    constexpr int kCols = D / kGroups;
     uint8_t* out = static_cast<uint8_t*>(p.dq) +
-                   ((size_t)(w.start + (valid ? q : 0)) * p.Hq + w.h) * (size_t)D * 2 + x * D;
+                   ((size_t)(w.start + (valid ? q : 0)) * p.Hq + w.h) * (size_t)D * 2 + x * kCols * 2;
+    uint32_t v[kCols];
+    if constexpr (kCols == 32) {
+        ptx::tmem_ld32_sync(tl + 256 + x * kCols, v);
+    } else {
+        tmem_ld16_sync(tl + 256 + x * kCols, v);
+    }
+    uint32_t pk[kCols / 2];
 #pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-        uint32_t v[32];
-        ptx::tmem_ld32_sync(tl + 256 + x * (D / 2) + cc * 32, v);
-        uint32_t pk[16];
+    for (int i = 0; i < kCols / 2; ++i)
+        pk[i] = ptx::pack_bf16x2(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
+    if (valid) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            pk[i] = ptx::pack_bf16x2(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
-        if (valid) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                ptx::st_global_v4(out + cc * 64 + u * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
+        for (int u = 0; u < kCols / 8; ++u)
+            ptx::st_global_v4(out + u * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
     }
 }
 
@@ -739,7 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    if (warp < 8) {
+    if (warp < kElemWarps) {
         dq_elementwise<D, STAGES>(w, p, tmem, sbase, abort_flag);
     } else if (warp == kWarpProducer) {
         dq_producer<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, &tm_do, sbase, abort_flag);
