@@ -14,8 +14,8 @@
 
 namespace {
 
-constexpr int kStages128 = 2;  // Q + dO (dK/dV kernel) or K + V (dQ kernel): 64 KB per stage
-constexpr int kStages64 = 4;
+constexpr int kStages128 = 4;  // 64-row Q + dO (dK/dV kernel) or K + V (dQ kernel): 32 KB per stage
+constexpr int kStages64 = 8;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -40,14 +40,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, cols] bf16 in boxes of 128 rows x 64 columns (128 bytes), 128-byte
-// swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+// [rows, cols] bf16 in boxes of box_rows rows x 64 columns (128 bytes),
+// 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estride[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -86,9 +86,13 @@ int prepare_device() {
     return ATTN_OK;
 }
 
+// Maps with 128-row boxes (the stationary tiles) and 64-row boxes (the streamed steps).
+struct Maps {
+    CUtensorMap q, k, v, dout, q64, k64, v64, dout64;
+};
+
 template <int D, int S>
-int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-           const attn::bwd::BwdParams& p, long long tokens, cudaStream_t s) {
+int launch(const Maps& m, const attn::bwd::BwdParams& p, long long tokens, cudaStream_t s) {
     using namespace attn::bwd;
     const long long rows = tokens * p.Hq;
     long long dblocks = (rows + 7) / 8;
@@ -97,10 +101,10 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
     attn_bwd_dsum<D><<<(unsigned)dblocks, 256, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     const unsigned dkv_grid = (unsigned)((long long)p.n_blocks * p.B * p.Hkv);
-    attn_bwd_dkv<D, S><<<dkv_grid, kThreads, DkvLayout<D, S>::kDynamicBytes, s>>>(mq, mk, mv, mdo, p);
+    attn_bwd_dkv<D, S><<<dkv_grid, kThreads, DkvLayout<D, S>::kDynamicBytes, s>>>(m.q64, m.k, m.v, m.dout64, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     const unsigned dq_grid = (unsigned)((long long)p.n_blocks * p.B * p.Hq);
-    attn_bwd_dq<D, S><<<dq_grid, kThreads, DqLayout<D, S>::kDynamicBytes, s>>>(mq, mk, mv, mdo, p);
+    attn_bwd_dq<D, S><<<dq_grid, kThreads, DqLayout<D, S>::kDynamicBytes, s>>>(m.q, m.k64, m.v64, m.dout, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -146,11 +150,12 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     int rc = prepare_device();
     if (rc != ATTN_OK) return rc;
 
-    CUtensorMap mq, mk, mv, mdo;
-    if (!make_map(&mq, q, (uint64_t)tokens, (uint64_t)Hq * d) ||
-        !make_map(&mk, k, (uint64_t)tokens, (uint64_t)Hkv * d) ||
-        !make_map(&mv, v, (uint64_t)tokens, (uint64_t)Hkv * d) ||
-        !make_map(&mdo, dout, (uint64_t)tokens, (uint64_t)Hq * d))
+    Maps mp;
+    const uint64_t T = (uint64_t)tokens, cq = (uint64_t)Hq * d, ck = (uint64_t)Hkv * d;
+    if (!make_map(&mp.q, q, T, cq, 128) || !make_map(&mp.k, k, T, ck, 128) ||
+        !make_map(&mp.v, v, T, ck, 128) || !make_map(&mp.dout, dout, T, cq, 128) ||
+        !make_map(&mp.q64, q, T, cq, 64) || !make_map(&mp.k64, k, T, ck, 64) ||
+        !make_map(&mp.v64, v, T, ck, 64) || !make_map(&mp.dout64, dout, T, cq, 64))
         return ATTN_ERR_CUDA;
 
     attn::bwd::BwdParams p;
@@ -176,6 +181,5 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     p.wait_limit_ns = kWaitLimitNs;
     if ((long long)p.n_blocks * B * Hq > 0x7fffffffLL) return ATTN_ERR_SHAPE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return d == 128 ? launch<128, kStages128>(mq, mk, mv, mdo, p, tokens, s)
-                    : launch<64, kStages64>(mq, mk, mv, mdo, p, tokens, s);
+    return d == 128 ? launch<128, kStages128>(mp, p, tokens, s) : launch<64, kStages64>(mp, p, tokens, s);
 }

@@ -9,22 +9,26 @@
 //
 //   attn_bwd_dsum    D_i for every (row, head), fp32, one warp per row.
 //   attn_bwd_dkv     one CTA per (sequence, key/value head, 128-key block).  K and
-//                    V stay in shared memory; the Q and dO tiles of every query
-//                    head of the group and every query block that sees the keys
-//                    stream through a 2-stage ring.  Per query block:
+//                    V stay in shared memory; the Q and dO tiles (64 rows) of every
+//                    query head of the group and every query step that sees the
+//                    keys stream through a 4-stage ring.  Per 64-row step:
 //                      S^T = K Q^T, dP^T = V dO^T      (tcgen05, both from smem)
 //                      P^T, dS^T                        (16 warps, fp32 -> bf16)
 //                      dV += P^T dO, dK += dS^T Q       (A from tensor memory)
-//                    dK and dV stay in tensor memory for the whole loop, so each
-//                    key row is written once, already summed over the group.
+//                    S^T / dP^T have two buffers: the products of step t + 1 run
+//                    while the elementwise warps work on step t.  dK and dV stay in
+//                    tensor memory for the whole loop, so each key row is written
+//                    once, already summed over the group.
 //   attn_bwd_dq      one CTA per (sequence, query head, 128-row block), over the
-//                    key blocks the rows see: S = Q K^T, dP = dO V^T, dS, then
-//                    dQ += dS K.  dQ stays in tensor memory; no atomics.
+//                    64-key steps the rows see: S = Q K^T, dP = dO V^T, dS, then
+//                    dQ += dS K, S / dP double-buffered the same way.  dQ stays in
+//                    tensor memory; no atomics.
 //
-// Tensor memory (512 columns): dkv: S^T [0,128), dP^T [128,256), dV [256,256+d),
-// dK [384,384+d); dq: S [0,128), dP [128,256), dQ [256,256+d).  The bf16 P^T /
-// dS^T (dS) are written into the upper 64 columns of their fp32 source region
-// once every column group has read it, and the next product reads them there.
+// Tensor memory (512 columns): dkv: S^T buffers [0,64) [64,128), dP^T buffers
+// [128,192) [192,256), dV [256,256+d), dK [384,384+d); dq: S [0,64) [64,128),
+// dP [128,192) [192,256), dQ [256,256+d).  The bf16 P^T / dS^T (dS) of a step go
+// to the upper 32 columns of their fp32 buffer once every column group has read
+// it, and the next product reads them there.
 //
 // Warps: 0-15 elementwise (column group x = warp / 4 takes the tile's columns
 // [32x, 32x + 32); warp w % 4 its 32 tensor-memory lanes: four warps per
@@ -44,17 +48,19 @@ namespace bwd {
 // Device status word of the backward kernels (read by attn_device_status).
 __device__ int g_bwd_status;
 
-constexpr int kBM = 128;  // query rows per block
-constexpr int kBN = 128;  // keys per block
+constexpr int kBM = 128;  // query rows of a dq CTA
+constexpr int kBN = 128;  // keys of a dkv CTA
+constexpr int kStep = 64; // rows (dkv) or keys (dq) streamed per step
 constexpr int kElemWarps = 16;              // 4 column groups x 4 lane quadrants
 constexpr int kGroups = kElemWarps / 4;      // column groups
-constexpr int kGroupCols = 128 / kGroups;    // columns of a step per group
+constexpr int kGroupCols = kStep / kGroups;  // columns of a step per group (16)
 constexpr int kWarpProducer = kElemWarps;
 constexpr int kWarpMma = kElemWarps + 1;
 constexpr int kThreads = (kElemWarps + 2) * 32;
 constexpr int kElemThreads = kElemWarps * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kBoxBytes = 128 * 128;  // one TMA box: 128 rows x 128 bytes
+constexpr uint32_t kBox128 = 128 * 128;  // TMA box of a 128-row tile: 128 rows x 128 bytes
+constexpr uint32_t kBox64 = 64 * 128;    // TMA box of a 64-row step tile
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdParams {
@@ -151,47 +157,48 @@ __device__ __forceinline__ bool visible(const BwdParams& p, int q, int k) {
     return (p.left < 0 || k >= q - p.left) && (p.right < 0 || k <= q + p.right);
 }
 
-// Every (query, key) pair of query block m x key block n is inside the
-// sequence and visible: no element mask needed.
-__device__ __forceinline__ bool block_full(const BwdParams& p, int m, int n, int len) {
-    const long long q0 = (long long)m * kBM, k0 = (long long)n * kBN;
-    if (q0 + kBM > len || k0 + kBN > len) return false;
-    if (p.left >= 0 && k0 < q0 + kBM - 1 - p.left) return false;
-    if (p.right >= 0 && k0 + kBN - 1 > q0 + p.right) return false;
+// Every (query, key) pair of queries [q0, q0 + nq) x keys [k0, k0 + nk) is
+// inside the sequence and visible: no element mask needed.
+__device__ __forceinline__ bool block_full(const BwdParams& p, long long q0, int nq, long long k0, int nk,
+                                           int len) {
+    if (q0 + nq > len || k0 + nk > len) return false;
+    if (p.left >= 0 && k0 < q0 + nq - 1 - p.left) return false;
+    if (p.right >= 0 && k0 + nk - 1 > q0 + p.right) return false;
     return true;
 }
 
-// Query blocks [m_lo, m_hi) that see some key of key block n.
-__device__ __forceinline__ void query_blocks(const BwdParams& p, int n, int len, int& m_lo, int& m_hi) {
+// 64-row query steps [m_lo, m_hi) that see some key of the 128-key block n.
+__device__ __forceinline__ void query_steps(const BwdParams& p, int n, int len, int& m_lo, int& m_hi) {
     const long long k0 = (long long)n * kBN;
     long long lo = p.right >= 0 ? k0 - p.right : 0;
     long long hi = p.left >= 0 ? k0 + kBN + p.left : len;  // exclusive
     if (lo < 0) lo = 0;
     if (hi > len) hi = len;
-    m_lo = (int)(lo / kBM);
-    m_hi = hi > lo ? (int)((hi + kBM - 1) / kBM) : m_lo;
+    m_lo = (int)(lo / kStep);
+    m_hi = hi > lo ? (int)((hi + kStep - 1) / kStep) : m_lo;
 }
 
-// Key blocks [n_lo, n_hi) that some row of query block m sees.
-__device__ __forceinline__ void key_blocks(const BwdParams& p, int m, int len, int& n_lo, int& n_hi) {
+// 64-key steps [n_lo, n_hi) that some row of the 128-row query block m sees.
+__device__ __forceinline__ void key_steps(const BwdParams& p, int m, int len, int& n_lo, int& n_hi) {
     const long long q0 = (long long)m * kBM;
     long long lo = p.left >= 0 ? q0 - p.left : 0;
     long long hi = p.right >= 0 ? q0 + kBM + p.right : len;  // exclusive
     if (lo < 0) lo = 0;
     if (hi > len) hi = len;
-    n_lo = (int)(lo / kBN);
-    n_hi = hi > lo ? (int)((hi + kBN - 1) / kBN) : n_lo;
+    n_lo = (int)(lo / kStep);
+    n_hi = hi > lo ? (int)((hi + kStep - 1) / kStep) : n_lo;
 }
 
-// K-major operand (rows x d, 128-byte swizzle, 64-column boxes 16 KB apart):
-// descriptor of the 16-column step kk.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
-    return ptx::smem_desc_sw128(tile + (kk / 4) * kBoxBytes + (kk % 4) * 32, 16, 1024);
+// K-major operand (rows x d, 128-byte swizzle, 64-column boxes `box` bytes
+// apart): descriptor of the 16-column step kk.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk, uint32_t box) {
+    return ptx::smem_desc_sw128(tile + (kk / 4) * box + (kk % 4) * 32, 16, 1024);
 }
 
-// MN-major B operand ([K rows, N = d columns], N contiguous): the 16-row step kk.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) {
-    return ptx::smem_desc_sw128(tile + kk * 2048, kBoxBytes, 1024);
+// MN-major B operand ([K rows, N = d columns], N contiguous, the two 64-column
+// halves `box` bytes apart): the 16-row step kk.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, uint32_t box) {
+    return ptx::smem_desc_sw128(tile + kk * 2048, box, 1024);
 }
 
 // ------------------------------------------------------------ D = rowsum(dO * O)
@@ -238,34 +245,44 @@ __global__ void __launch_bounds__(256) attn_bwd_dsum(const BwdParams p) {
 }
 
 // ------------------------------------------------------------ dK, dV
+// Tensor memory: S^T buffer b at [64b, 64b + 64), dP^T buffer b at
+// [128 + 64b, 128 + 64b + 64) (b = step & 1), dV [256, 256 + d), dK [384, 384 + d).
+// P^T / dS^T of a step (64 queries -> 32 packed columns) go to the upper half of
+// their buffer.  The products of step t + 1 are issued before the hand-off of
+// step t, so they run while the elementwise warps work on step t.
 template <int D, int STAGES>
 struct DkvLayout {
-    static constexpr uint32_t kTile = kBN * D * 2;
+    static constexpr uint32_t kTileK = kBN * D * 2;    // K or V: 128 keys
+    static constexpr uint32_t kTileQ = kStep * D * 2;  // Q or dO: 64 rows
     static constexpr uint32_t kK = 0;
-    static constexpr uint32_t kV = kTile;
-    static constexpr uint32_t kRing = 2 * kTile;
-    static constexpr uint32_t kSlot = 2 * kTile + 1024;  // Q, dO, lse2[128], D[128]
+    static constexpr uint32_t kV = kTileK;
+    static constexpr uint32_t kRing = 2 * kTileK;
+    static constexpr uint32_t kSlot = (2 * kTileQ + 2 * kStep * 4 + 1023) / 1024 * 1024;  // Q, dO, lse2, D
     static constexpr uint32_t kBar = kRing + STAGES * kSlot;
-    // kv_loaded, slot_full[S], slot_empty[S], st_full, p_ready, done
-    static constexpr uint32_t kNumBars = 4 + 2 * STAGES;
+    // kv_loaded, slot_full[S], slot_empty[S], st_full[2], p_ready[2], done
+    static constexpr uint32_t kNumBars = 6 + 2 * STAGES;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 
     static __device__ __forceinline__ uint32_t q(uint32_t base, int s) { return base + kRing + s * kSlot; }
-    static __device__ __forceinline__ uint32_t dout(uint32_t base, int s) { return q(base, s) + kTile; }
-    static __device__ __forceinline__ uint32_t stats(uint32_t base, int s) { return q(base, s) + 2 * kTile; }
+    static __device__ __forceinline__ uint32_t dout(uint32_t base, int s) { return q(base, s) + kTileQ; }
+    static __device__ __forceinline__ uint32_t stats(uint32_t base, int s) { return q(base, s) + 2 * kTileQ; }
     static __device__ __forceinline__ uint32_t bar_kv(uint32_t base) { return base + kBar; }
     static __device__ __forceinline__ uint32_t bar_full(uint32_t base, int s) { return base + kBar + 8u * (1 + s); }
     static __device__ __forceinline__ uint32_t bar_empty(uint32_t base, int s) {
         return base + kBar + 8u * (1 + STAGES + s);
     }
-    static __device__ __forceinline__ uint32_t bar_st(uint32_t base) { return base + kBar + 8u * (1 + 2 * STAGES); }
-    static __device__ __forceinline__ uint32_t bar_p(uint32_t base) { return base + kBar + 8u * (2 + 2 * STAGES); }
-    static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (3 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_st(uint32_t base, int b) {
+        return base + kBar + 8u * (1 + 2 * STAGES + b);
+    }
+    static __device__ __forceinline__ uint32_t bar_p(uint32_t base, int b) {
+        return base + kBar + 8u * (3 + 2 * STAGES + b);
+    }
+    static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (5 + 2 * STAGES); }
 };
 
-// The (query head, query block) steps of a key block, in loop order.
+// The (query head, 64-row query step) steps of a key block, in loop order.
 struct DkvWork {
     int b, g, n, start, len, m_lo, m_hi, steps;
 };
@@ -273,7 +290,7 @@ struct DkvWork {
 __device__ __forceinline__ DkvWork dkv_work(const BwdParams& p) {
     DkvWork w;
     const int per_n = p.B * p.Hkv;
-    w.n = blockIdx.x / per_n;  // key block 0 (the most query blocks under a causal mask) first
+    w.n = blockIdx.x / per_n;  // key block 0 (the most query steps under a causal mask) first
     const int rem = blockIdx.x % per_n;
     w.b = rem / p.Hkv;
     w.g = rem % p.Hkv;
@@ -285,27 +302,27 @@ __device__ __forceinline__ DkvWork dkv_work(const BwdParams& p) {
         w.m_lo = w.m_hi = 0;
         return w;
     }
-    query_blocks(p, w.n, w.len, w.m_lo, w.m_hi);
+    query_steps(p, w.n, w.len, w.m_lo, w.m_hi);
     w.steps = p.group * (w.m_hi - w.m_lo);
     return w;
 }
 
 template <int D, int STAGES>
-__device__ __forceinline__ void dkv_producer(const DkvWork& w, const BwdParams& p, const CUtensorMap* tm_q,
+__device__ __forceinline__ void dkv_producer(const DkvWork& w, const BwdParams& p, const CUtensorMap* tm_q64,
                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                             const CUtensorMap* tm_do, uint32_t sbase,
+                                             const CUtensorMap* tm_do64, uint32_t sbase,
                                              volatile int* abort_flag, uint8_t* smem) {
     using L = DkvLayout<D, STAGES>;
     constexpr int kBoxes = D / 64;
     const int lane = threadIdx.x % 32;
     const uint64_t pol_kv = ptx::policy_evict_first();
     const uint64_t pol_q = ptx::policy_evict_last();  // reread by the other key blocks
-    ptx::mbar_arrive_expect_tx_elect(L::bar_kv(sbase), 2 * L::kTile);
+    ptx::mbar_arrive_expect_tx_elect(L::bar_kv(sbase), 2 * L::kTileK);
 #pragma unroll
     for (int bx = 0; bx < kBoxes; ++bx) {
-        ptx::tma_load_2d_elect(sbase + L::kK + bx * kBoxBytes, tm_k, L::bar_kv(sbase), w.g * D + bx * 64,
+        ptx::tma_load_2d_elect(sbase + L::kK + bx * kBox128, tm_k, L::bar_kv(sbase), w.g * D + bx * 64,
                                w.start + w.n * kBN, pol_kv);
-        ptx::tma_load_2d_elect(sbase + L::kV + bx * kBoxBytes, tm_v, L::bar_kv(sbase), w.g * D + bx * 64,
+        ptx::tma_load_2d_elect(sbase + L::kV + bx * kBox128, tm_v, L::bar_kv(sbase), w.g * D + bx * 64,
                                w.start + w.n * kBN, pol_kv);
     }
     const int nm = w.m_hi - w.m_lo;
@@ -315,27 +332,27 @@ __device__ __forceinline__ void dkv_producer(const DkvWork& w, const BwdParams& 
         if (!warp_wait(L::bar_empty(sbase, s), ((t / STAGES) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
         const int h = w.g * p.group + t / nm;
         const int m = w.m_lo + t % nm;
-        ptx::mbar_arrive_expect_tx_elect(L::bar_full(sbase, s), 2 * L::kTile);
+        ptx::mbar_arrive_expect_tx_elect(L::bar_full(sbase, s), 2 * L::kTileQ);
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
-            ptx::tma_load_2d_elect(L::q(sbase, s) + bx * kBoxBytes, tm_q, L::bar_full(sbase, s),
-                                   h * D + bx * 64, w.start + m * kBM, pol_q);
-            ptx::tma_load_2d_elect(L::dout(sbase, s) + bx * kBoxBytes, tm_do, L::bar_full(sbase, s),
-                                   h * D + bx * 64, w.start + m * kBM, pol_q);
+            ptx::tma_load_2d_elect(L::q(sbase, s) + bx * kBox64, tm_q64, L::bar_full(sbase, s),
+                                   h * D + bx * 64, w.start + m * kStep, pol_q);
+            ptx::tma_load_2d_elect(L::dout(sbase, s) + bx * kBox64, tm_do64, L::bar_full(sbase, s),
+                                   h * D + bx * 64, w.start + m * kStep, pol_q);
         }
-        // lse2 and D of the block's 128 rows (0 past the sequence's end)
+        // lse2 and D of the step's 64 rows (0 past the sequence's end)
         float* st = reinterpret_cast<float*>(smem + (L::stats(sbase, s) - sbase));
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int i = m * kBM + lane * 4 + e;
+        for (int e = 0; e < kStep / 32; ++e) {
+            const int i = m * kStep + lane * (kStep / 32) + e;
             float l2 = 0.0f, dd = 0.0f;
             if (i < w.len) {
                 const size_t idx = stat_index(p, w.b, h, w.start, i);
                 l2 = p.lse[idx] * kLog2e;
                 dd = p.dsum[idx];
             }
-            st[lane * 4 + e] = l2;
-            st[kBM + lane * 4 + e] = dd;
+            st[lane * (kStep / 32) + e] = l2;
+            st[kStep + lane * (kStep / 32) + e] = dd;
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(L::bar_full(sbase, s));
@@ -351,34 +368,43 @@ template <int D, int STAGES>
 __device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, uint32_t tmem, uint32_t sbase,
                                         volatile int* abort_flag) {
     using L = DkvLayout<D, STAGES>;
-    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kBN, kBM, false, false);  // M keys, N queries
-    constexpr uint32_t kIdG = ptx::idesc_bf16_f32(kBN, D, false, true);     // M keys, N = d
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kBN, kStep, false, false);  // M keys, N = 64 queries
+    constexpr uint32_t kIdG = ptx::idesc_bf16_f32(kBN, D, false, true);       // M keys, N = d
     const unsigned long long lim = p.wait_limit_ns;
     bool ok = warp_wait(L::bar_kv(sbase), 0, abort_flag, lim);
     ptx::tc_fence_after_sync();
-    for (int t = 0; ok && t < w.steps; ++t) {
+    // S^T(t) and dP^T(t) into buffer t & 1
+    auto issue_st = [&](int t) -> bool {
         const int s = t % STAGES;
-        if (!(ok = warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim))) break;
+        if (!warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim)) return false;
         ptx::tc_fence_after_sync();
-        const uint32_t qt = L::q(sbase, s), dot = L::dout(sbase, s);
+        const uint32_t buf = (t & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)  // S^T = K Q^T
-            ptx::mma_ss_elect(tmem, kmajor_desc(sbase + L::kK, kk), kmajor_desc(qt, kk), kIdS, kk > 0 ? 1u : 0u);
+            ptx::mma_ss_elect(tmem + buf, kmajor_desc(sbase + L::kK, kk, kBox128),
+                              kmajor_desc(L::q(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)  // dP^T = V dO^T
-            ptx::mma_ss_elect(tmem + 128, kmajor_desc(sbase + L::kV, kk), kmajor_desc(dot, kk), kIdS,
-                              kk > 0 ? 1u : 0u);
-        ptx::tc_commit_elect(L::bar_st(sbase));
-        if (!(ok = warp_wait(L::bar_p(sbase), t & 1, abort_flag, lim))) break;
+            ptx::mma_ss_elect(tmem + 128 + buf, kmajor_desc(sbase + L::kV, kk, kBox128),
+                              kmajor_desc(L::dout(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
+        ptx::tc_commit_elect(L::bar_st(sbase, t & 1));
+        return true;
+    };
+    if (ok && w.steps > 0) ok = issue_st(0);
+    for (int t = 0; ok && t < w.steps; ++t) {
+        if (t + 1 < w.steps && !(ok = issue_st(t + 1))) break;
+        if (!(ok = warp_wait(L::bar_p(sbase, t & 1), (t >> 1) & 1, abort_flag, lim))) break;
         ptx::tc_fence_after_sync();
+        const int s = t % STAGES;
+        const uint32_t buf = (t & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk)  // dV += P^T dO
-            ptx::mma_ts_elect(tmem + 256, tmem + 64 + kk * 8, mnmajor_desc(dot, kk), kIdG,
-                              (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kStep / 16; ++kk)  // dV += P^T dO
+            ptx::mma_ts_elect(tmem + 256, tmem + buf + 32 + kk * 8, mnmajor_desc(L::dout(sbase, s), kk, kBox64),
+                              kIdG, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk)  // dK += dS^T Q
-            ptx::mma_ts_elect(tmem + 384, tmem + 192 + kk * 8, mnmajor_desc(qt, kk), kIdG,
-                              (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kStep / 16; ++kk)  // dK += dS^T Q
+            ptx::mma_ts_elect(tmem + 384, tmem + 128 + buf + 32 + kk * 8, mnmajor_desc(L::q(sbase, s), kk, kBox64),
+                              kIdG, (t > 0 || kk > 0) ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_empty(sbase, s));
     }
     ptx::tc_commit_elect(L::bar_done(sbase));
@@ -386,7 +412,7 @@ __device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, ui
 }
 
 // One thread = one key row (tensor-memory lane); column group x = warp / 4
-// takes query columns [32x, 32x + 32) of every step.
+// takes query columns [16x, 16x + 16) of every 64-row step.
 template <int D, int STAGES>
 __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParams& p, uint32_t tmem,
                                                 uint32_t sbase, uint8_t* smem, volatile int* abort_flag) {
@@ -402,47 +428,45 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
     const unsigned long long lim = p.wait_limit_ns;
     bool ok = true;
     for (int t = 0; t < w.steps; ++t) {
-        if (!(ok = warp_wait(L::bar_st(sbase), t & 1, abort_flag, lim))) break;
-        ptx::tc_fence_after_sync();
         const int s = t % STAGES;
+        const uint32_t buf = (t & 1) * 64;
+        if (!(ok = warp_wait(L::bar_st(sbase, t & 1), (t >> 1) & 1, abort_flag, lim))) break;
+        // the statistics were written by the producer before this slot's arrival
+        if (!(ok = warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
         const int m = w.m_lo + t % nm;
         const float* st = reinterpret_cast<const float*>(smem + (L::stats(sbase, s) - sbase));
-        const bool full = block_full(p, m, w.n, w.len);
-        uint32_t pp[kGroupCols / 2], pd[kGroupCols / 2];
+        const bool full = block_full(p, (long long)m * kStep, kStep, (long long)w.n * kBN, kBN, w.len);
+        const int col0 = kGroupCols * x;
+        uint32_t sv[16], dv[16], pp[8], pd[8];
+        tmem_ld16_sync(tl + buf + col0, sv);
+        tmem_ld16_sync(tl + 128 + buf + col0, dv);
 #pragma unroll
-        for (int c = 0; c < kGroupCols / 16; ++c) {
-            const int col0 = kGroupCols * x + 16 * c;
-            uint32_t sv[16], dv[16];
-            tmem_ld16_sync(tl + col0, sv);
-            tmem_ld16_sync(tl + 128 + col0, dv);
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                const int ql = col0 + i;
-                const float2 l2 = *reinterpret_cast<const float2*>(st + ql);
-                const float2 dd = *reinterpret_cast<const float2*>(st + kBM + ql);
-                float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2.x));
-                float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2.y));
-                if (!full) {
-                    const int q = m * kBM + ql;
-                    if (!(q < w.len && key < w.len && visible(p, q, key))) p0 = 0.0f;
-                    if (!(q + 1 < w.len && key < w.len && visible(p, q + 1, key))) p1 = 0.0f;
-                }
-                const float d0 = p0 * (__uint_as_float(dv[i]) - dd.x);
-                const float d1 = p1 * (__uint_as_float(dv[i + 1]) - dd.y);
-                pp[c * 8 + i / 2] = ptx::pack_bf16x2(p0, p1);
-                pd[c * 8 + i / 2] = ptx::pack_bf16x2(d0, d1);
+        for (int i = 0; i < 16; i += 2) {
+            const int ql = col0 + i;
+            const float2 l2 = *reinterpret_cast<const float2*>(st + ql);
+            const float2 dd = *reinterpret_cast<const float2*>(st + kStep + ql);
+            float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2.x));
+            float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2.y));
+            if (!full) {
+                const int q = m * kStep + ql;
+                if (!(q < w.len && key < w.len && visible(p, q, key))) p0 = 0.0f;
+                if (!(q + 1 < w.len && key < w.len && visible(p, q + 1, key))) p1 = 0.0f;
             }
+            pp[i / 2] = ptx::pack_bf16x2(p0, p1);
+            pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd.x),
+                                         p1 * (__uint_as_float(dv[i + 1]) - dd.y));
         }
         // every group has read its S^T / dP^T columns before any overwrites the
         // upper halves with P^T / dS^T
         ptx::tc_fence_before_sync();
         elem_sync();
         ptx::tc_fence_after_sync();
-        ptx::tmem_st16(tl + 64 + (kGroupCols / 2) * x, pp);
-        ptx::tmem_st16(tl + 192 + (kGroupCols / 2) * x, pd);
+        ptx::tmem_st8(tl + buf + 32 + 8 * x, pp);
+        ptx::tmem_st8(tl + 128 + buf + 32 + 8 * x, pd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(L::bar_p(sbase));
+        ptx::mbar_arrive(L::bar_p(sbase, t & 1));
     }
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
@@ -473,8 +497,8 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
 
 template <int D, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    attn_bwd_dkv(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
                  const BwdParams p) {
     using L = DkvLayout<D, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -492,15 +516,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(L::bar_full(sbase, s), 2);  // expect_tx arrival + statistics arrival
             ptx::mbar_init(L::bar_empty(sbase, s), 1);
         }
-        ptx::mbar_init(L::bar_st(sbase), 1);
-        ptx::mbar_init(L::bar_p(sbase), kElemThreads);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(L::bar_st(sbase, b), 1);
+            ptx::mbar_init(L::bar_p(sbase, b), kElemThreads);
+        }
         ptx::mbar_init(L::bar_done(sbase), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
-        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_q64);
         ptx::prefetch_tensormap(&tm_k);
         ptx::prefetch_tensormap(&tm_v);
-        ptx::prefetch_tensormap(&tm_do);
+        ptx::prefetch_tensormap(&tm_do64);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
@@ -513,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kElemWarps) {
         dkv_elementwise<D, STAGES>(w, p, tmem, sbase, smem, abort_flag);
     } else if (warp == kWarpProducer) {
-        dkv_producer<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, &tm_do, sbase, abort_flag, smem);
+        dkv_producer<D, STAGES>(w, p, &tm_q64, &tm_k, &tm_v, &tm_do64, sbase, abort_flag, smem);
     } else {
         dkv_mma<D, STAGES>(w, p, tmem, sbase, abort_flag);
     }
@@ -524,30 +550,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------ dQ
+// Tensor memory: S buffer b at [64b, 64b + 64), dP buffer b at
+// [128 + 64b, 128 + 64b + 64), dQ [256, 256 + d); dS (64 keys -> 32 packed
+// columns) goes to the upper half of its S buffer.
 template <int D, int STAGES>
 struct DqLayout {
-    static constexpr uint32_t kTile = kBM * D * 2;
+    static constexpr uint32_t kTileQ = kBM * D * 2;    // Q or dO: 128 rows
+    static constexpr uint32_t kTileK = kStep * D * 2;  // K or V: 64 keys
     static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kDO = kTile;
-    static constexpr uint32_t kRing = 2 * kTile;
-    static constexpr uint32_t kSlot = 2 * kTile;  // K, V
+    static constexpr uint32_t kDO = kTileQ;
+    static constexpr uint32_t kRing = 2 * kTileQ;
+    static constexpr uint32_t kSlot = 2 * kTileK;  // K, V
     static constexpr uint32_t kBar = kRing + STAGES * kSlot;
-    // q_loaded, slot_full[S], slot_empty[S], st_full, ds_ready, done
-    static constexpr uint32_t kNumBars = 4 + 2 * STAGES;
+    // q_loaded, slot_full[S], slot_empty[S], st_full[2], ds_ready[2], done
+    static constexpr uint32_t kNumBars = 6 + 2 * STAGES;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 
     static __device__ __forceinline__ uint32_t k(uint32_t base, int s) { return base + kRing + s * kSlot; }
-    static __device__ __forceinline__ uint32_t v(uint32_t base, int s) { return k(base, s) + kTile; }
+    static __device__ __forceinline__ uint32_t v(uint32_t base, int s) { return k(base, s) + kTileK; }
     static __device__ __forceinline__ uint32_t bar_q(uint32_t base) { return base + kBar; }
     static __device__ __forceinline__ uint32_t bar_full(uint32_t base, int s) { return base + kBar + 8u * (1 + s); }
     static __device__ __forceinline__ uint32_t bar_empty(uint32_t base, int s) {
         return base + kBar + 8u * (1 + STAGES + s);
     }
-    static __device__ __forceinline__ uint32_t bar_st(uint32_t base) { return base + kBar + 8u * (1 + 2 * STAGES); }
-    static __device__ __forceinline__ uint32_t bar_ds(uint32_t base) { return base + kBar + 8u * (2 + 2 * STAGES); }
-    static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (3 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_st(uint32_t base, int b) {
+        return base + kBar + 8u * (1 + 2 * STAGES + b);
+    }
+    static __device__ __forceinline__ uint32_t bar_ds(uint32_t base, int b) {
+        return base + kBar + 8u * (3 + 2 * STAGES + b);
+    }
+    static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (5 + 2 * STAGES); }
 };
 
 struct DqWork {
@@ -557,7 +591,7 @@ struct DqWork {
 __device__ __forceinline__ DqWork dq_work(const BwdParams& p) {
     DqWork w;
     const int per_m = p.B * p.Hq;
-    w.m = p.n_blocks - 1 - blockIdx.x / per_m;  // latest rows (most key blocks, causal) first
+    w.m = p.n_blocks - 1 - blockIdx.x / per_m;  // latest rows (most key steps, causal) first
     const int rem = blockIdx.x % per_m;
     w.b = rem / p.Hq;
     w.h = rem % p.Hq;
@@ -569,37 +603,37 @@ __device__ __forceinline__ DqWork dq_work(const BwdParams& p) {
         w.n_lo = w.n_hi = 0;
         return w;
     }
-    key_blocks(p, w.m, w.len, w.n_lo, w.n_hi);
+    key_steps(p, w.m, w.len, w.n_lo, w.n_hi);
     return w;
 }
 
 template <int D, int STAGES>
 __device__ __forceinline__ void dq_producer(const DqWork& w, const BwdParams& p, const CUtensorMap* tm_q,
-                                            const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                            const CUtensorMap* tm_k64, const CUtensorMap* tm_v64,
                                             const CUtensorMap* tm_do, uint32_t sbase, volatile int* abort_flag) {
     using L = DqLayout<D, STAGES>;
     constexpr int kBoxes = D / 64;
     const uint64_t pol_q = ptx::policy_evict_first();
     const uint64_t pol_kv = ptx::policy_evict_last();
-    ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * L::kTile);
+    ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * L::kTileQ);
 #pragma unroll
     for (int bx = 0; bx < kBoxes; ++bx) {
-        ptx::tma_load_2d_elect(sbase + L::kQ + bx * kBoxBytes, tm_q, L::bar_q(sbase), w.h * D + bx * 64,
+        ptx::tma_load_2d_elect(sbase + L::kQ + bx * kBox128, tm_q, L::bar_q(sbase), w.h * D + bx * 64,
                                w.start + w.m * kBM, pol_q);
-        ptx::tma_load_2d_elect(sbase + L::kDO + bx * kBoxBytes, tm_do, L::bar_q(sbase), w.h * D + bx * 64,
+        ptx::tma_load_2d_elect(sbase + L::kDO + bx * kBox128, tm_do, L::bar_q(sbase), w.h * D + bx * 64,
                                w.start + w.m * kBM, pol_q);
     }
     int issued = 0;
     for (int n = w.n_lo; n < w.n_hi; ++n) {
         const int t = n - w.n_lo, s = t % STAGES;
         if (!warp_wait(L::bar_empty(sbase, s), ((t / STAGES) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
-        ptx::mbar_arrive_expect_tx_elect(L::bar_full(sbase, s), 2 * L::kTile);
+        ptx::mbar_arrive_expect_tx_elect(L::bar_full(sbase, s), 2 * L::kTileK);
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
-            ptx::tma_load_2d_elect(L::k(sbase, s) + bx * kBoxBytes, tm_k, L::bar_full(sbase, s),
-                                   w.g * D + bx * 64, w.start + n * kBN, pol_kv);
-            ptx::tma_load_2d_elect(L::v(sbase, s) + bx * kBoxBytes, tm_v, L::bar_full(sbase, s),
-                                   w.g * D + bx * 64, w.start + n * kBN, pol_kv);
+            ptx::tma_load_2d_elect(L::k(sbase, s) + bx * kBox64, tm_k64, L::bar_full(sbase, s),
+                                   w.g * D + bx * 64, w.start + n * kStep, pol_kv);
+            ptx::tma_load_2d_elect(L::v(sbase, s) + bx * kBox64, tm_v64, L::bar_full(sbase, s),
+                                   w.g * D + bx * 64, w.start + n * kStep, pol_kv);
         }
         ++issued;
     }
@@ -613,29 +647,38 @@ template <int D, int STAGES>
 __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint32_t tmem, uint32_t sbase,
                                        volatile int* abort_flag) {
     using L = DqLayout<D, STAGES>;
-    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kBM, kBN, false, false);
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kBM, kStep, false, false);  // M queries, N = 64 keys
     constexpr uint32_t kIdG = ptx::idesc_bf16_f32(kBM, D, false, true);
     const unsigned long long lim = p.wait_limit_ns;
+    const int steps = w.n_hi - w.n_lo;
     bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
     ptx::tc_fence_after_sync();
-    for (int n = w.n_lo; ok && n < w.n_hi; ++n) {
-        const int t = n - w.n_lo, s = t % STAGES;
-        if (!(ok = warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim))) break;
+    auto issue_st = [&](int t) -> bool {  // S(t) and dP(t) into buffer t & 1
+        const int s = t % STAGES;
+        if (!warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim)) return false;
         ptx::tc_fence_after_sync();
-        const uint32_t kt = L::k(sbase, s), vt = L::v(sbase, s);
+        const uint32_t buf = (t & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)  // S = Q K^T
-            ptx::mma_ss_elect(tmem, kmajor_desc(sbase + L::kQ, kk), kmajor_desc(kt, kk), kIdS, kk > 0 ? 1u : 0u);
+            ptx::mma_ss_elect(tmem + buf, kmajor_desc(sbase + L::kQ, kk, kBox128),
+                              kmajor_desc(L::k(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)  // dP = dO V^T
-            ptx::mma_ss_elect(tmem + 128, kmajor_desc(sbase + L::kDO, kk), kmajor_desc(vt, kk), kIdS,
-                              kk > 0 ? 1u : 0u);
-        ptx::tc_commit_elect(L::bar_st(sbase));
-        if (!(ok = warp_wait(L::bar_ds(sbase), t & 1, abort_flag, lim))) break;
+            ptx::mma_ss_elect(tmem + 128 + buf, kmajor_desc(sbase + L::kDO, kk, kBox128),
+                              kmajor_desc(L::v(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
+        ptx::tc_commit_elect(L::bar_st(sbase, t & 1));
+        return true;
+    };
+    if (ok && steps > 0) ok = issue_st(0);
+    for (int t = 0; ok && t < steps; ++t) {
+        if (t + 1 < steps && !(ok = issue_st(t + 1))) break;
+        if (!(ok = warp_wait(L::bar_ds(sbase, t & 1), (t >> 1) & 1, abort_flag, lim))) break;
         ptx::tc_fence_after_sync();
+        const int s = t % STAGES;
+        const uint32_t buf = (t & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)  // dQ += dS K
-            ptx::mma_ts_elect(tmem + 256, tmem + 64 + kk * 8, mnmajor_desc(kt, kk), kIdG,
+        for (int kk = 0; kk < kStep / 16; ++kk)  // dQ += dS K
+            ptx::mma_ts_elect(tmem + 256, tmem + buf + 32 + kk * 8, mnmajor_desc(L::k(sbase, s), kk, kBox64), kIdG,
                               (t > 0 || kk > 0) ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_empty(sbase, s));
     }
@@ -644,7 +687,7 @@ __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint
 }
 
 // One thread = one query row; column group x = warp / 4 takes key columns
-// [32x, 32x + 32).
+// [16x, 16x + 16) of every 64-key step.
 template <int D, int STAGES>
 __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams& p, uint32_t tmem,
                                                uint32_t sbase, volatile int* abort_flag) {
@@ -667,36 +710,32 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
     bool ok = true;
     for (int n = w.n_lo; n < w.n_hi; ++n) {
         const int t = n - w.n_lo;
-        if (!(ok = warp_wait(L::bar_st(sbase), t & 1, abort_flag, lim))) break;
+        const uint32_t buf = (t & 1) * 64;
+        if (!(ok = warp_wait(L::bar_st(sbase, t & 1), (t >> 1) & 1, abort_flag, lim))) break;
         ptx::tc_fence_after_sync();
-        const bool full = block_full(p, w.m, n, w.len);
-        uint32_t pd[kGroupCols / 2];
+        const bool full = block_full(p, (long long)w.m * kBM, kBM, (long long)n * kStep, kStep, w.len);
+        const int col0 = kGroupCols * x;
+        uint32_t sv[16], dv[16], pd[8];
+        tmem_ld16_sync(tl + buf + col0, sv);
+        tmem_ld16_sync(tl + 128 + buf + col0, dv);
 #pragma unroll
-        for (int c = 0; c < kGroupCols / 16; ++c) {
-            const int col0 = kGroupCols * x + 16 * c;
-            uint32_t sv[16], dv[16];
-            tmem_ld16_sync(tl + col0, sv);
-            tmem_ld16_sync(tl + 128 + col0, dv);
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2));
-                float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2));
-                if (!full) {
-                    const int k = n * kBN + col0 + i;
-                    if (!(valid && k < w.len && visible(p, q, k))) p0 = 0.0f;
-                    if (!(valid && k + 1 < w.len && visible(p, q, k + 1))) p1 = 0.0f;
-                }
-                pd[c * 8 + i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd),
-                                                     p1 * (__uint_as_float(dv[i + 1]) - dd));
+        for (int i = 0; i < 16; i += 2) {
+            float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2));
+            float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2));
+            if (!full) {
+                const int k = n * kStep + col0 + i;
+                if (!(valid && k < w.len && visible(p, q, k))) p0 = 0.0f;
+                if (!(valid && k + 1 < w.len && visible(p, q, k + 1))) p1 = 0.0f;
             }
+            pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd), p1 * (__uint_as_float(dv[i + 1]) - dd));
         }
         ptx::tc_fence_before_sync();
         elem_sync();
         ptx::tc_fence_after_sync();
-        ptx::tmem_st16(tl + 64 + (kGroupCols / 2) * x, pd);
+        ptx::tmem_st8(tl + buf + 32 + 8 * x, pd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(L::bar_ds(sbase));
+        ptx::mbar_arrive(L::bar_ds(sbase, t & 1));
     }
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
@@ -724,8 +763,8 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
 
 template <int D, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    attn_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k64,
+                const __grid_constant__ CUtensorMap tm_v64, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p) {
     using L = DqLayout<D, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -743,14 +782,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(L::bar_full(sbase, s), 1);
             ptx::mbar_init(L::bar_empty(sbase, s), 1);
         }
-        ptx::mbar_init(L::bar_st(sbase), 1);
-        ptx::mbar_init(L::bar_ds(sbase), kElemThreads);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(L::bar_st(sbase, b), 1);
+            ptx::mbar_init(L::bar_ds(sbase, b), kElemThreads);
+        }
         ptx::mbar_init(L::bar_done(sbase), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_q);
-        ptx::prefetch_tensormap(&tm_k);
-        ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_k64);
+        ptx::prefetch_tensormap(&tm_v64);
         ptx::prefetch_tensormap(&tm_do);
     }
     if (warp == kWarpMma) {
@@ -764,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kElemWarps) {
         dq_elementwise<D, STAGES>(w, p, tmem, sbase, abort_flag);
     } else if (warp == kWarpProducer) {
-        dq_producer<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, &tm_do, sbase, abort_flag);
+        dq_producer<D, STAGES>(w, p, &tm_q, &tm_k64, &tm_v64, &tm_do, sbase, abort_flag);
     } else {
         dq_mma<D, STAGES>(w, p, tmem, sbase, abort_flag);
     }
