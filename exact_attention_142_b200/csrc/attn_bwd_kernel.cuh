@@ -26,9 +26,9 @@
 //
 // Tensor memory (512 columns): dkv: S^T buffers [0,64) [64,128), dP^T buffers
 // [128,192) [192,256), dV [256,256+d), dK [384,384+d); dq: S [0,64) [64,128),
-// dP [128,192) [192,256), dQ [256,256+d).  The bf16 P^T / dS^T (dS) of a step go
-// to the upper 32 columns of their fp32 buffer once every column group has read
-// it, and the next product reads them there.
+// dP [128,192) [192,256), dQ [256,256+d).  Each column group writes the bf16
+// P^T / dS^T (dS) of its 16 columns into the first 8 of those same columns, and
+// the next products read them there (one K-step per 16 columns).
 //
 // Warps: 0-15 elementwise (column group x = warp / 4 takes the tile's columns
 // [32x, 32x + 32); warp w % 4 its 32 tensor-memory lanes: four warps per
@@ -126,10 +126,6 @@ __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
-}
-
-__device__ __forceinline__ void elem_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kElemThreads) : "memory");
 }
 
 struct Seq {
@@ -247,9 +243,11 @@ __global__ void __launch_bounds__(256) attn_bwd_dsum(const BwdParams p) {
 // ------------------------------------------------------------ dK, dV
 // Tensor memory: S^T buffer b at [64b, 64b + 64), dP^T buffer b at
 // [128 + 64b, 128 + 64b + 64) (b = step & 1), dV [256, 256 + d), dK [384, 384 + d).
-// P^T / dS^T of a step (64 queries -> 32 packed columns) go to the upper half of
-// their buffer.  The products of step t + 1 are issued before the hand-off of
-// step t, so they run while the elementwise warps work on step t.
+// The bf16 P^T / dS^T of queries [16c, 16c + 16) of a step (8 packed columns) go
+// to the first 8 of that buffer's columns 16c.. (the ones their column group just
+// read), and the products read K-step c there.  The products of step t + 1 are
+// issued before the hand-off of step t, so they run while the elementwise warps
+// work on step t.
 template <int D, int STAGES>
 struct DkvLayout {
     static constexpr uint32_t kTileK = kBN * D * 2;    // K or V: 128 keys
@@ -398,12 +396,12 @@ __device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, ui
         const int s = t % STAGES;
         const uint32_t buf = (t & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < kStep / 16; ++kk)  // dV += P^T dO
-            ptx::mma_ts_elect(tmem + 256, tmem + buf + 32 + kk * 8, mnmajor_desc(L::dout(sbase, s), kk, kBox64),
+        for (int kk = 0; kk < kStep / 16; ++kk)  // dV += P^T dO  (P^T of queries 16kk.. at column 16kk)
+            ptx::mma_ts_elect(tmem + 256, tmem + buf + 16 * kk, mnmajor_desc(L::dout(sbase, s), kk, kBox64),
                               kIdG, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kStep / 16; ++kk)  // dK += dS^T Q
-            ptx::mma_ts_elect(tmem + 384, tmem + 128 + buf + 32 + kk * 8, mnmajor_desc(L::q(sbase, s), kk, kBox64),
+            ptx::mma_ts_elect(tmem + 384, tmem + 128 + buf + 16 * kk, mnmajor_desc(L::q(sbase, s), kk, kBox64),
                               kIdG, (t > 0 || kk > 0) ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_empty(sbase, s));
     }
@@ -457,13 +455,10 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
             pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd.x),
                                          p1 * (__uint_as_float(dv[i + 1]) - dd.y));
         }
-        // every group has read its S^T / dP^T columns before any overwrites the
-        // upper halves with P^T / dS^T
-        ptx::tc_fence_before_sync();
-        elem_sync();
-        ptx::tc_fence_after_sync();
-        ptx::tmem_st8(tl + buf + 32 + 8 * x, pp);
-        ptx::tmem_st8(tl + 128 + buf + 32 + 8 * x, pd);
+        // P^T / dS^T of these 16 queries go to the first 8 of the 16 columns this
+        // thread has just read: no other group reads them, so no barrier is needed
+        ptx::tmem_st8(tl + buf + col0, pp);
+        ptx::tmem_st8(tl + 128 + buf + col0, pd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_p(sbase, t & 1));
@@ -551,8 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------ dQ
 // Tensor memory: S buffer b at [64b, 64b + 64), dP buffer b at
-// [128 + 64b, 128 + 64b + 64), dQ [256, 256 + d); dS (64 keys -> 32 packed
-// columns) goes to the upper half of its S buffer.
+// [128 + 64b, 128 + 64b + 64), dQ [256, 256 + d); dS of keys [16c, 16c + 16)
+// (8 packed columns) goes to the first 8 of the S buffer's columns 16c...
 template <int D, int STAGES>
 struct DqLayout {
     static constexpr uint32_t kTileQ = kBM * D * 2;    // Q or dO: 128 rows
@@ -677,8 +672,8 @@ __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint
         const int s = t % STAGES;
         const uint32_t buf = (t & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < kStep / 16; ++kk)  // dQ += dS K
-            ptx::mma_ts_elect(tmem + 256, tmem + buf + 32 + kk * 8, mnmajor_desc(L::k(sbase, s), kk, kBox64), kIdG,
+        for (int kk = 0; kk < kStep / 16; ++kk)  // dQ += dS K  (dS of keys 16kk.. at column 16kk)
+            ptx::mma_ts_elect(tmem + 256, tmem + buf + 16 * kk, mnmajor_desc(L::k(sbase, s), kk, kBox64), kIdG,
                               (t > 0 || kk > 0) ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_empty(sbase, s));
     }
@@ -729,10 +724,7 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
             }
             pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd), p1 * (__uint_as_float(dv[i + 1]) - dd));
         }
-        ptx::tc_fence_before_sync();
-        elem_sync();
-        ptx::tc_fence_after_sync();
-        ptx::tmem_st8(tl + buf + 32 + 8 * x, pd);
+        ptx::tmem_st8(tl + buf + col0, pd);  // into the columns this thread has just read
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_ds(sbase, t & 1));
