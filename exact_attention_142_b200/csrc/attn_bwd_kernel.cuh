@@ -435,30 +435,33 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
         const int m = w.m_lo + t % nm;
         const float* st = reinterpret_cast<const float*>(smem + (L::stats(sbase, s) - sbase));
         const bool full = block_full(p, (long long)m * kStep, kStep, (long long)w.n * kBN, kBN, w.len);
-        const int col0 = kGroupCols * x;
-        uint32_t sv[16], dv[16], pp[8], pd[8];
-        tmem_ld16_sync(tl + buf + col0, sv);
-        tmem_ld16_sync(tl + 128 + buf + col0, dv);
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            const int ql = col0 + i;
-            const float2 l2 = *reinterpret_cast<const float2*>(st + ql);
-            const float2 dd = *reinterpret_cast<const float2*>(st + kStep + ql);
-            float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2.x));
-            float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2.y));
-            if (!full) {
-                const int q = m * kStep + ql;
-                if (!(q < w.len && key < w.len && visible(p, q, key))) p0 = 0.0f;
-                if (!(q + 1 < w.len && key < w.len && visible(p, q + 1, key))) p1 = 0.0f;
+        for (int c = 0; c < kGroupCols / 16; ++c) {
+            const int col0 = kGroupCols * x + 16 * c;
+            uint32_t sv[16], dv[16], pp[8], pd[8];
+            tmem_ld16_sync(tl + buf + col0, sv);
+            tmem_ld16_sync(tl + 128 + buf + col0, dv);
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const int ql = col0 + i;
+                const float2 l2 = *reinterpret_cast<const float2*>(st + ql);
+                const float2 dd = *reinterpret_cast<const float2*>(st + kStep + ql);
+                float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2.x));
+                float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2.y));
+                if (!full) {
+                    const int q = m * kStep + ql;
+                    if (!(q < w.len && key < w.len && visible(p, q, key))) p0 = 0.0f;
+                    if (!(q + 1 < w.len && key < w.len && visible(p, q + 1, key))) p1 = 0.0f;
+                }
+                pp[i / 2] = ptx::pack_bf16x2(p0, p1);
+                pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd.x),
+                                             p1 * (__uint_as_float(dv[i + 1]) - dd.y));
             }
-            pp[i / 2] = ptx::pack_bf16x2(p0, p1);
-            pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd.x),
-                                         p1 * (__uint_as_float(dv[i + 1]) - dd.y));
+            // P^T / dS^T of these 16 queries go to the first 8 of the 16 columns this
+            // thread has just read: no other group reads them, so no barrier is needed
+            ptx::tmem_st8(tl + buf + col0, pp);
+            ptx::tmem_st8(tl + 128 + buf + col0, pd);
         }
-        // P^T / dS^T of these 16 queries go to the first 8 of the 16 columns this
-        // thread has just read: no other group reads them, so no barrier is needed
-        ptx::tmem_st8(tl + buf + col0, pp);
-        ptx::tmem_st8(tl + 128 + buf + col0, pd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_p(sbase, t & 1));
@@ -466,16 +469,19 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
     ptx::tc_fence_after_sync();
-    // groups 0, 1 store the two halves of dV's columns, groups 2, 3 of dK's (times the scale)
+    // the 2d output columns (dV then dK) are split evenly over the column groups
+    // (dK times the scale)
+    constexpr int kOutCols = 2 * D / kGroups;
     const bool store = key < w.len;
-    const bool is_k = x >= 2;
-    const int half = x & 1;
+    const int c_first = x * kOutCols;  // in [0, 2d)
+    const bool is_k = c_first >= D;
+    const int c_in = c_first % D;
     const float mul = is_k ? p.scale : 1.0f;
     uint8_t* out = static_cast<uint8_t*>(is_k ? p.dk : p.dv) +
-                   ((size_t)(w.start + (store ? key : 0)) * p.Hkv + w.g) * (size_t)D * 2 + half * D;
-    const uint32_t src = tl + (is_k ? 384u : 256u) + half * (D / 2);
+                   ((size_t)(w.start + (store ? key : 0)) * p.Hkv + w.g) * (size_t)D * 2 + c_in * 2;
+    const uint32_t src = tl + (is_k ? 384u : 256u) + c_in;
 #pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
+    for (int cc = 0; cc < kOutCols / 32; ++cc) {
         uint32_t v[32];
         ptx::tmem_ld32_sync(src + cc * 32, v);
         uint32_t pk[16];
@@ -709,22 +715,26 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
         if (!(ok = warp_wait(L::bar_st(sbase, t & 1), (t >> 1) & 1, abort_flag, lim))) break;
         ptx::tc_fence_after_sync();
         const bool full = block_full(p, (long long)w.m * kBM, kBM, (long long)n * kStep, kStep, w.len);
-        const int col0 = kGroupCols * x;
-        uint32_t sv[16], dv[16], pd[8];
-        tmem_ld16_sync(tl + buf + col0, sv);
-        tmem_ld16_sync(tl + 128 + buf + col0, dv);
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2));
-            float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2));
-            if (!full) {
-                const int k = n * kStep + col0 + i;
-                if (!(valid && k < w.len && visible(p, q, k))) p0 = 0.0f;
-                if (!(valid && k + 1 < w.len && visible(p, q, k + 1))) p1 = 0.0f;
+        for (int c = 0; c < kGroupCols / 16; ++c) {
+            const int col0 = kGroupCols * x + 16 * c;
+            uint32_t sv[16], dv[16], pd[8];
+            tmem_ld16_sync(tl + buf + col0, sv);
+            tmem_ld16_sync(tl + 128 + buf + col0, dv);
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                float p0 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -l2));
+                float p1 = ptx::ex2_approx(fmaf(__uint_as_float(sv[i + 1]), sl2, -l2));
+                if (!full) {
+                    const int k = n * kStep + col0 + i;
+                    if (!(valid && k < w.len && visible(p, q, k))) p0 = 0.0f;
+                    if (!(valid && k + 1 < w.len && visible(p, q, k + 1))) p1 = 0.0f;
+                }
+                pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd),
+                                             p1 * (__uint_as_float(dv[i + 1]) - dd));
             }
-            pd[i / 2] = ptx::pack_bf16x2(p0 * (__uint_as_float(dv[i]) - dd), p1 * (__uint_as_float(dv[i + 1]) - dd));
+            ptx::tmem_st8(tl + buf + col0, pd);  // into the columns this thread has just read
         }
-        ptx::tmem_st8(tl + buf + col0, pd);  // into the columns this thread has just read
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_ds(sbase, t & 1));
@@ -732,24 +742,22 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
     ptx::tc_fence_after_sync();
-    // group x stores columns [x * D/4, (x + 1) * D/4) of dQ (times the scale)
+    // group x stores columns [x * d / groups, (x + 1) * d / groups) of dQ (times the scale)
     constexpr int kCols = D / kGroups;
     uint8_t* out = static_cast<uint8_t*>(p.dq) +
                    ((size_t)(w.start + (valid ? q : 0)) * p.Hq + w.h) * (size_t)D * 2 + x * kCols * 2;
-    uint32_t v[kCols];
-    if constexpr (kCols == 32) {
-        ptx::tmem_ld32_sync(tl + 256 + x * kCols, v);
-    } else {
-        tmem_ld16_sync(tl + 256 + x * kCols, v);
-    }
-    uint32_t pk[kCols / 2];
 #pragma unroll
-    for (int i = 0; i < kCols / 2; ++i)
-        pk[i] = ptx::pack_bf16x2(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
-    if (valid) {
+    for (int c = 0; c < kCols / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16_sync(tl + 256 + x * kCols + 16 * c, v);
+        uint32_t pk[8];
 #pragma unroll
-        for (int u = 0; u < kCols / 8; ++u)
-            ptx::st_global_v4(out + u * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        for (int i = 0; i < 8; ++i)
+            pk[i] = ptx::pack_bf16x2(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
+        if (valid) {
+            ptx::st_global_v4(out + c * 32, pk[0], pk[1], pk[2], pk[3]);
+            ptx::st_global_v4(out + c * 32 + 16, pk[4], pk[5], pk[6], pk[7]);
+        }
     }
 }
 
