@@ -144,6 +144,9 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
 }
 
+// One CTA per tile pair; running CTAs take over the pairs of CTAs that have
+// not started (the kernel's persistent schedule), so only about one CTA per
+// SM ever runs.
 template <int D, int STAGES, bool ACC>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
            long long units, cudaStream_t stream) {

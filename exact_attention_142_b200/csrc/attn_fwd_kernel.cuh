@@ -61,6 +61,8 @@ constexpr float kLog2e = 1.442695040888963407f;
 // Register split after launch (384 threads x 168 = 64512 registers):
 // 128 x (216 + 216 + 72) = 64512.
 constexpr uint32_t kRegsSoftmax = 216;
+// Readers of the unit queue: the MMA warp and the eight softmax warps.
+constexpr uint32_t kUnitReaders = 9;
 constexpr uint32_t kRegsOther = 72;
 
 // One in kPolyPeriod groups of four weights takes its exponential from the
@@ -117,10 +119,13 @@ struct SmemLayout {
     static constexpr uint32_t kQ1 = kTileBytes;
     static constexpr uint32_t kKV = 2 * kTileBytes;
     static constexpr uint32_t kBar = kKV + STAGES * kTileBytes;
-    // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final
-    static constexpr uint32_t kNumBars = 8 + 2 * STAGES;
+    // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
+    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2]
+    static constexpr uint32_t kNumBars = 16 + 2 * STAGES;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem address, abort flag
-    static constexpr uint32_t kBytes = kMisc + 16;
+    static constexpr uint32_t kClcResp = kMisc + 16;        // launch-control response (16 B)
+    static constexpr uint32_t kUnitQ = kClcResp + 16;       // unit queue: two ints
+    static constexpr uint32_t kBytes = kUnitQ + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // room to align the base to 1 KB
 
     static __device__ __forceinline__ uint32_t bar_q(uint32_t base) { return base + kBar; }
@@ -142,7 +147,23 @@ struct SmemLayout {
     static __device__ __forceinline__ uint32_t bar_mma_final(uint32_t base) {
         return base + kBar + 8u * (7 + 2 * STAGES);
     }
+    static __device__ __forceinline__ uint32_t bar_q_empty(uint32_t base) {
+        return base + kBar + 8u * (8 + 2 * STAGES);
+    }
+    static __device__ __forceinline__ uint32_t bar_o_free(uint32_t base, int x) {
+        return base + kBar + 8u * (9 + 2 * STAGES + x);
+    }
+    static __device__ __forceinline__ uint32_t bar_clc(uint32_t base) {
+        return base + kBar + 8u * (11 + 2 * STAGES);
+    }
+    static __device__ __forceinline__ uint32_t bar_unit_full(uint32_t base, int slot) {
+        return base + kBar + 8u * (12 + 2 * STAGES + slot);
+    }
+    static __device__ __forceinline__ uint32_t bar_unit_empty(uint32_t base, int slot) {
+        return base + kBar + 8u * (14 + 2 * STAGES + slot);
+    }
 };
+
 
 // Wait for an mbarrier phase with a time limit.  On expiry the block-wide
 // abort flag is raised and the device status word records the timeout; once
@@ -181,6 +202,21 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity,
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned long long limit_ns) {
     return __all_sync(0xffffffffu, bounded_wait(bar, parity, abort_flag, limit_ns));
+}
+
+// Entry n of the CTA's unit queue (filled by the producer warp): the next tile
+// pair with rows to compute, or -1 once the grid's work is exhausted (or the
+// block aborted).  Called by a whole warp; lane 0 releases the slot.
+// Only n mod 4 matters (slot and phase).
+template <class L>
+__device__ __forceinline__ int unit_take(uint32_t sbase, uint32_t n, volatile int* abort_flag,
+                                         unsigned long long limit_ns) {
+    const int slot = n & 1;
+    if (!warp_wait(L::bar_unit_full(sbase, slot), (n >> 1) & 1, abort_flag, limit_ns)) return -1;
+    const int u = ptx::ld_volatile_smem(sbase + L::kUnitQ + 4 * slot);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(L::bar_unit_empty(sbase, slot));
+    return u;
 }
 
 // The two query tiles of one CTA and the key blocks each of them needs.
@@ -252,48 +288,103 @@ __device__ __forceinline__ bool tile_active_at(const TilePair& w, int x, int j) 
 }
 
 // ---------------------------------------------------------------- producer
+// Persistent, varlen-aware schedule.  The grid holds one CTA per tile pair in
+// heaviest-first order.  A running CTA starts with its own pair; when the
+// producer has issued every load of a pair it takes the next pending pair by
+// cancelling the launch of a CTA that has not started (cluster launch
+// control), skipping pairs with no rows (packed sequences shorter than the
+// longest), and passes it to the MMA and softmax warps through a two-entry
+// queue in shared memory.  Pairs are thus handed out greedily in the same
+// order as by the hardware's block scheduler, while the next pair's Q load
+// and first products overlap the previous pair's epilogue.
 template <int D, int STAGES>
-__device__ __forceinline__ void producer_role(const TilePair& w, const FwdParams& p,
-                                              const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                                              const CUtensorMap* tm_v, uint32_t sbase,
-                                              volatile int* abort_flag) {
+__device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              uint32_t sbase, volatile int* abort_flag) {
     using L = SmemLayout<D, STAGES>;
     constexpr int kBoxes = D / 64;
+    const unsigned long long lim = p.wait_limit_ns;
     const uint64_t pol_q = ptx::policy_evict_first();
     const uint64_t pol_kv = ptx::policy_evict_last();
-
-    ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * L::kTileBytes);
-    for (int x = 0; x < 2; ++x) {
-#pragma unroll
-        for (int bx = 0; bx < kBoxes; ++bx)
-            ptx::tma_load_2d_elect(sbase + (x ? L::kQ1 : L::kQ0) + bx * L::kBoxBytes, tm_q,
-                             L::bar_q(sbase), w.h[x] * D + bx * 64, w.start + w.r0[x], pol_q);
-    }
-
-    int issued = 0;
+    const uint32_t resp = sbase + L::kClcResp;
+    int issued = 0;      // K/V ring loads
+    int units = 0;       // pairs whose Q was loaded
+    int published = 0;   // unit queue entries written
+    int requests = 0;    // launch-control requests answered
+    bool pending = false;  // a request whose answer has not been seen
+    bool more = true;      // false after a request that cancelled nothing
+    int cand = blockIdx.x;
     bool ok = true;
-    for (int j = w.ulo; j < w.uhi && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv) {
-            const int s = issued % STAGES;
-            const uint32_t ph = (issued / STAGES) & 1;
-            if (!warp_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, p.wait_limit_ns)) {
-                ok = false;
-                break;
+
+    // The next pair with rows, or -1.
+    auto next_unit = [&]() -> int {
+        while (true) {
+            if (cand >= 0) {
+                const TilePair w = decode_pair(cand, p);
+                const int u = cand;
+                cand = -1;
+                if (w.active[0] || w.active[1]) return u;
             }
-            ptx::mbar_arrive_expect_tx_elect(L::bar_kv_full(sbase, s), L::kTileBytes);
+            if (!more) return -1;
+            ptx::fence_proxy_async_smem();  // the last response was read before it is rewritten
+            __syncwarp();
+            ptx::clc_try_cancel_elect(resp, L::bar_clc(sbase));
+            pending = true;
+            if (!warp_wait(L::bar_clc(sbase), requests & 1, abort_flag, lim)) {
+                ok = false;
+                return -1;
+            }
+            pending = false;
+            ++requests;
+            cand = ptx::clc_query_x(resp);
+            if (cand < 0) more = false;
+        }
+    };
+    auto publish = [&](int u) -> bool {
+        const int slot = published & 1;
+        if (!warp_wait(L::bar_unit_empty(sbase, slot), ((published >> 1) & 1) ^ 1, abort_flag, lim))
+            return false;
+        if ((threadIdx.x & 31) == 0) ptx::st_volatile_smem(sbase + L::kUnitQ + 4 * slot, u);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(L::bar_unit_full(sbase, slot));
+        ++published;
+        return true;
+    };
+
+    int u = next_unit();
+    while (ok) {
+        if (!(ok = publish(u)) || u < 0) break;
+        const TilePair w = decode_pair(u, p);
+        // the previous pair's score products have finished reading Q
+        if (units > 0 && !(ok = warp_wait(L::bar_q_empty(sbase), (units - 1) & 1, abort_flag, lim))) break;
+        ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * L::kTileBytes);
+        for (int x = 0; x < 2; ++x) {
 #pragma unroll
             for (int bx = 0; bx < kBoxes; ++bx)
-                ptx::tma_load_2d_elect(sbase + L::kKV + s * L::kTileBytes + bx * L::kBoxBytes,
-                                 kv ? tm_v : tm_k, L::bar_kv_full(sbase, s), w.g * D + bx * 64,
-                                 w.start + j * kBN, pol_kv);
-            ++issued;
+                ptx::tma_load_2d_elect(sbase + (x ? L::kQ1 : L::kQ0) + bx * L::kBoxBytes, tm_q, L::bar_q(sbase),
+                                       w.h[x] * D + bx * 64, w.start + w.r0[x], pol_q);
         }
+        ++units;
+        for (int j = w.ulo; j < w.uhi && ok; ++j) {
+            for (int kv = 0; kv < 2; ++kv) {
+                const int s = issued % STAGES;
+                const uint32_t ph = (issued / STAGES) & 1;
+                if (!(ok = warp_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, lim))) break;
+                ptx::mbar_arrive_expect_tx_elect(L::bar_kv_full(sbase, s), L::kTileBytes);
+#pragma unroll
+                for (int bx = 0; bx < kBoxes; ++bx)
+                    ptx::tma_load_2d_elect(sbase + L::kKV + s * L::kTileBytes + bx * L::kBoxBytes, kv ? tm_v : tm_k,
+                                           L::bar_kv_full(sbase, s), w.g * D + bx * 64, w.start + j * kBN, pol_kv);
+                ++issued;
+            }
+        }
+        if (ok) u = next_unit();
     }
-    // Every copy issued must have landed before the block may exit.
-    drain_wait(L::bar_q(sbase), 0, p.wait_limit_ns);
+    // Every copy and request issued must have landed before the block may exit.
+    if (pending) drain_wait(L::bar_clc(sbase), requests & 1, lim);
+    if (units > 0) drain_wait(L::bar_q(sbase), (units - 1) & 1, lim);
     const int first = issued > STAGES ? issued - STAGES : 0;
-    for (int i = first; i < issued; ++i)
-        drain_wait(L::bar_kv_full(sbase, i % STAGES), (i / STAGES) & 1, p.wait_limit_ns);
+    for (int i = first; i < issued; ++i) drain_wait(L::bar_kv_full(sbase, i % STAGES), (i / STAGES) & 1, lim);
 }
 
 // ---------------------------------------------------------------- MMA issuer
@@ -333,70 +424,97 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
 }
 
 template <int D, int STAGES>
-__device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, uint32_t tmem,
-                                         uint32_t sbase, volatile int* abort_flag) {
+__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint32_t sbase,
+                                         volatile int* abort_flag) {
     using L = SmemLayout<D, STAGES>;
     const unsigned long long lim = p.wait_limit_ns;
-    bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
-    ptx::tc_fence_after_sync();
-    int pc[2] = {0, 0};
-    bool first[2] = {true, true};
-    // Issue order per key block j:  S0(j), PV1(j-1), S1(j), PV0(j).  Each
-    // softmax group then has the two products of the other tile to hide its
-    // exponentials behind.  S_x(j) overwrites the P_x(j-1) columns only after
-    // PV_x(j-1) was issued; tcgen05 MMAs from one thread execute in order.
-    for (int j = w.ulo; ok && j < w.uhi; ++j) {
-        const int kidx = 2 * (j - w.ulo), vidx = kidx + 1;
-        const int ks = kidx % STAGES, vs = vidx % STAGES;
-        if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (kidx / STAGES) & 1, abort_flag, lim)))
-            break;
+    // Phase bits, kept in one word (this warp runs with few registers):
+    enum : uint32_t {
+        kPc = 1u,          // << x: parity of the P hand-offs consumed for tile x
+        kPending = 4u,     // << x: O of tile x handed to an epilogue not yet released
+        kFreed = 16u,      // << x: parity of the o_free phases consumed for tile x
+        kFirst = 64u,      // << x: the next PV of tile x starts a fresh accumulator
+        kQ = 256u,         // parity of the Q loads consumed
+        kUnitShift = 9u,   // bits 9-10: unit queue index mod 4
+    };
+    uint32_t f = 0;
+    int ring = 0;  // K/V ring slots consumed
+    bool ok = true;
+    // Waits for p_ready of tile x; before the first PV of a pair also for the
+    // previous pair's epilogue to have read O.
+    auto pv_ready = [&](int x) -> bool {
+        if (!warp_wait(L::bar_p_ready(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
+        f ^= kPc << x;
+        if ((f & (kFirst << x)) && (f & (kPending << x))) {
+            if (!warp_wait(L::bar_o_free(sbase, x), (f >> (4 + x)) & 1u, abort_flag, lim)) return false;
+            f ^= (kFreed << x) | (kPending << x);
+        }
         ptx::tc_fence_after_sync();
-        if (tile_active_at(w, 0, j)) {
-            issue_qk<D, STAGES>(tmem, sbase, 0, ks);
-            ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
+        return true;
+    };
+    auto pv = [&](int x, int slot, bool last) {
+        issue_pv<D, STAGES>(tmem, sbase, x, slot, !(f & (kFirst << x)));
+        f &= ~(kFirst << x);
+        if (last) {
+            ptx::tc_commit_elect(L::bar_o_done(sbase, x));
+            f |= kPending << x;
         }
-        if (j > w.ulo) {
-            const int pvs = (vidx - 2) % STAGES;
-            if (tile_active_at(w, 1, j - 1)) {
-                if (!(ok = warp_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim)))
-                    break;
-                ++pc[1];
-                ptx::tc_fence_after_sync();
-                issue_pv<D, STAGES>(tmem, sbase, 1, pvs, !first[1]);
-                first[1] = false;
-                if (j - 1 == w.hi[1] - 1) ptx::tc_commit_elect(L::bar_o_done(sbase, 1));
-            }
-            ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
-        }
-        if (tile_active_at(w, 1, j)) {
-            issue_qk<D, STAGES>(tmem, sbase, 1, ks);
-            ptx::tc_commit_elect(L::bar_s_full(sbase, 1));
-        }
-        ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
-        if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), (vidx / STAGES) & 1, abort_flag, lim)))
-            break;
+    };
+    while (ok) {
+        const int u = unit_take<L>(sbase, (f >> kUnitShift) & 3u, abort_flag, lim);
+        f = (f & ~(3u << kUnitShift)) | ((((f >> kUnitShift) + 1u) & 3u) << kUnitShift);
+        if (u < 0) break;
+        const TilePair w = decode_pair(u, p);
+        const int lo0 = w.lo[0], hi0 = w.hi[0], lo1 = w.lo[1], hi1 = w.hi[1];  // empty when inactive
+        if (!(ok = warp_wait(L::bar_q(sbase), (f & kQ) ? 1u : 0u, abort_flag, lim))) break;
+        f ^= kQ;
+        f |= kFirst | (kFirst << 1);
         ptx::tc_fence_after_sync();
-        if (tile_active_at(w, 0, j)) {
-            if (!(ok = warp_wait(L::bar_p_ready(sbase, 0), pc[0] & 1, abort_flag, lim))) break;
-            ++pc[0];
+        // Issue order per key block j:  S0(j), PV1(j-1), S1(j), PV0(j).  Each
+        // softmax group then has the two products of the other tile to hide its
+        // exponentials behind.  S_x(j) overwrites the P_x(j-1) columns only after
+        // PV_x(j-1) was issued; tcgen05 MMAs from one thread execute in order.
+        for (int j = w.ulo; ok && j < w.uhi; ++j, ring += 2) {
+            const int ks = ring % STAGES, vs = (ring + 1) % STAGES;
+            if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (ring / STAGES) & 1, abort_flag, lim))) break;
             ptx::tc_fence_after_sync();
-            issue_pv<D, STAGES>(tmem, sbase, 0, vs, !first[0]);
-            first[0] = false;
-            if (j == w.hi[0] - 1) ptx::tc_commit_elect(L::bar_o_done(sbase, 0));
-        }
-    }
-    if (ok && w.uhi > w.ulo) {
-        const int j = w.uhi - 1;
-        const int vs = (2 * (j - w.ulo) + 1) % STAGES;
-        if (tile_active_at(w, 1, j)) {
-            ok = warp_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim);
-            if (ok) {
-                ptx::tc_fence_after_sync();
-                issue_pv<D, STAGES>(tmem, sbase, 1, vs, !first[1]);
-                ptx::tc_commit_elect(L::bar_o_done(sbase, 1));
+            if (j >= lo0 && j < hi0) {
+                issue_qk<D, STAGES>(tmem, sbase, 0, ks);
+                ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
+            }
+            if (j > w.ulo) {
+                const int pvs = (ring - 1) % STAGES;
+                if (j - 1 >= lo1 && j - 1 < hi1) {
+                    if (!(ok = pv_ready(1))) break;
+                    pv(1, pvs, j - 1 == hi1 - 1);
+                }
+                ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
+            }
+            if (j >= lo1 && j < hi1) {
+                issue_qk<D, STAGES>(tmem, sbase, 1, ks);
+                ptx::tc_commit_elect(L::bar_s_full(sbase, 1));
+            }
+            ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
+            if (j == w.uhi - 1) ptx::tc_commit_elect(L::bar_q_empty(sbase));  // last score products issued
+            if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), ((ring + 1) / STAGES) & 1, abort_flag, lim))) break;
+            ptx::tc_fence_after_sync();
+            if (j >= lo0 && j < hi0) {
+                if (!(ok = pv_ready(0))) break;
+                pv(0, vs, j == hi0 - 1);
             }
         }
-        ptx::tc_commit_elect(L::bar_kv_empty(sbase, vs));
+        if (!ok) break;
+        if (w.uhi > w.ulo) {
+            const int j = w.uhi - 1;
+            const int vs = (ring - 1) % STAGES;
+            if (j >= lo1 && j < hi1) {
+                if (!(ok = pv_ready(1))) break;
+                pv(1, vs, true);
+            }
+            ptx::tc_commit_elect(L::bar_kv_empty(sbase, vs));
+        } else {
+            ptx::tc_commit_elect(L::bar_q_empty(sbase));  // no products: Q is free
+        }
     }
     // All MMAs must be complete before tensor memory is released.
     ptx::tc_commit_elect(L::bar_mma_final(sbase));
@@ -409,17 +527,13 @@ __device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, 
 // accumulator's log-sum-exp) by the online-softmax rule (Step 3 applied to two
 // partial results; "Long context beyond a single GPU").
 template <int D, int STAGES, bool ACC>
-__device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams& p, int x,
+__device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams& p, int x,
                                              int warp_in_group, int lane, uint32_t tmem,
-                                             uint32_t sbase, volatile int* abort_flag) {
+                                             uint32_t sbase, volatile int* abort_flag, uint32_t& phases, int u) {
     using L = SmemLayout<D, STAGES>;
-    // Per-tile scalars (avoid dynamic indexing of the pair's small arrays).
-    const bool active = x ? w.active[1] : w.active[0];
-    if (!active) return;
     const int r0 = x ? w.r0[1] : w.r0[0];
     const int blk_lo = x ? w.lo[1] : w.lo[0];
     const int blk_hi = x ? w.hi[1] : w.hi[0];
-    const int h = x ? w.h[1] : w.h[0];
     const unsigned long long lim = p.wait_limit_ns;
     const int row = r0 + warp_in_group * 32 + lane;  // row within the sequence
     const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
@@ -442,9 +556,9 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
     bool ok = true;
 
     for (int j = blk_lo; j < blk_hi; ++j) {
-        ok = __all_sync(0xffffffffu,
-                        bounded_wait(L::bar_s_full(sbase, x), (j - blk_lo) & 1, abort_flag, lim));
+        ok = __all_sync(0xffffffffu, bounded_wait(L::bar_s_full(sbase, x), phases & 1u, abort_flag, lim));
         if (!ok) break;
+        phases ^= 1u;
         ptx::tc_fence_after_sync();
         uint32_t s[128];
         ptx::tmem_ld128_sync(t_s, s);
@@ -549,16 +663,21 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
         ptx::mbar_arrive(L::bar_p_ready(sbase, x));
     }
 
-    if (!ok) return;
+    if (!ok) return false;
     // Epilogue (Step 4 and 5): wait for the last PV product, divide once by the
     // sum, round to bf16, and store O and the log-sum-exp.
-    ok = __all_sync(0xffffffffu, bounded_wait(L::bar_o_done(sbase, x), 0, abort_flag, lim));
-    if (!ok) return;
+    ok = __all_sync(0xffffffffu, bounded_wait(L::bar_o_done(sbase, x), (phases >> 1) & 1u, abort_flag, lim));
+    if (!ok) return false;
     ptx::tc_fence_after_sync();
-    const bool store = row < w.len;
+    // The pair's indices again (recomputed rather than kept live through the loop).
+    int u_again = u;
+    asm volatile("" : "+r"(u_again));
+    const TilePair we = decode_pair(u_again, p);
+    const int h = x ? we.h[1] : we.h[0];
+    const bool store = row < we.len;
     if constexpr (ACC) {
-        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + w.start + (store ? row : 0)
-                                        : ((size_t)w.b * p.Hq + h) * p.N + (store ? row : 0);
+        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + (store ? row : 0)
+                                        : ((size_t)we.b * p.Hq + h) * p.N + (store ? row : 0);
         // both log-sum-exps in log2 units; weights relative to the larger one
         const float lse_new = l_sum > 0.0f ? m_ref + ptx::lg2_approx(l_sum) : -INFINITY;
         const float lse_old = store ? p.lse[idx] * kLog2e : -INFINITY;
@@ -570,7 +689,7 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
         const float inv_den = den > 0.0f ? 1.0f / den : 0.0f;
         const float a_old = w_old * inv_den;
         const float a_new = l_bf > 0.0f ? w_new * inv_den / l_bf : 0.0f;
-        float* acc = static_cast<float*>(p.o) + ((size_t)(w.start + (store ? row : 0)) * p.Hq + h) * (size_t)D;
+        float* acc = static_cast<float*>(p.o) + ((size_t)(we.start + (store ? row : 0)) * p.Hq + h) * (size_t)D;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
@@ -589,11 +708,13 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
             }
         }
         if (store) p.lse[idx] = den > 0.0f ? (mu + ptx::lg2_approx(den)) * kLn2 : -INFINITY;
-        return;
+        ptx::tc_fence_before_sync();
+        ptx::mbar_arrive(L::bar_o_free(sbase, x));
+        return true;
     }
     const float inv = l_bf > 0.0f ? 1.0f / l_bf : 0.0f;
     uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
-                    ((size_t)(w.start + (store ? row : 0)) * p.Hq + h) * (size_t)D * 2;
+                    ((size_t)(we.start + (store ? row : 0)) * p.Hq + h) * (size_t)D * 2;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -611,9 +732,31 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
     }
     if (store) {
         const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
-        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + w.start + row
-                                        : ((size_t)w.b * p.Hq + h) * p.N + row;
+        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + row
+                                        : ((size_t)we.b * p.Hq + h) * p.N + row;
         p.lse[idx] = lse;
+    }
+    // O has been read: the next unit's first PV of this tile may overwrite it
+    ptx::tc_fence_before_sync();
+    ptx::mbar_arrive(L::bar_o_free(sbase, x));
+    return true;
+}
+
+// The units of this CTA for one tile of the pair (tiles with no rows skipped).
+template <int D, int STAGES, bool ACC>
+__device__ __forceinline__ void softmax_role(const FwdParams& p, int x, int warp_in_group, int lane,
+                                             uint32_t tmem, uint32_t sbase, volatile int* abort_flag) {
+    // bit 0: s_full parity, bit 1: o_done parity, bits 2-3: unit queue index mod 4
+    uint32_t phases = 0;
+    while (true) {
+        const int u = unit_take<SmemLayout<D, STAGES>>(sbase, phases >> 2, abort_flag, p.wait_limit_ns);
+        phases = (phases + 4u) & 15u;
+        if (u < 0) break;
+        const TilePair w = decode_pair(u, p);
+        if (!(x ? w.active[1] : w.active[0])) continue;
+        if (!softmax_unit<D, STAGES, ACC>(w, p, x, warp_in_group, lane, tmem, sbase, abort_flag, phases, u))
+            return;
+        phases ^= 2u;
     }
 }
 
@@ -630,9 +773,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
 
-    const TilePair w = decode_pair(blockIdx.x, p);
-    if (!w.active[0] && !w.active[1]) return;  // uniform over the block
-
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -648,6 +788,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(L::bar_o_done(sbase, x), 1);
         }
         ptx::mbar_init(L::bar_mma_final(sbase), 1);
+        ptx::mbar_init(L::bar_q_empty(sbase), 1);
+        for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_o_free(sbase, x), 128);
+        ptx::mbar_init(L::bar_clc(sbase), 1);
+        for (int slot = 0; slot < 2; ++slot) {
+            ptx::mbar_init(L::bar_unit_full(sbase, slot), 1);
+            ptx::mbar_init(L::bar_unit_empty(sbase, slot), kUnitReaders);
+        }
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_q);
@@ -665,13 +812,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
-        softmax_role<D, STAGES, ACC>(w, p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
+        softmax_role<D, STAGES, ACC>(p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (warp == kWarpProducer) {
-            producer_role<D, STAGES>(w, p, &tm_q, &tm_k, &tm_v, sbase, abort_flag);
+            producer_role<D, STAGES>(p, &tm_q, &tm_k, &tm_v, sbase, abort_flag);
         } else if (warp == kWarpMma) {
-            mma_role<D, STAGES>(w, p, tmem, sbase, abort_flag);
+            mma_role<D, STAGES>(p, tmem, sbase, abort_flag);
         }
     }
 

@@ -404,5 +404,55 @@ __device__ __forceinline__ void st_global_v4(void* ptr, uint32_t a, uint32_t b, 
                  : "memory");
 }
 
+__device__ __forceinline__ int ld_volatile_smem(uint32_t addr) {
+    int v;
+    asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_volatile_smem(uint32_t addr, int v) {
+    asm volatile("st.volatile.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy ones (a TMA or launch-control write into the same bytes).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Cluster launch control (sm_100): ask the hardware to cancel the launch of a
+// CTA that has not started yet, so that this CTA can do its work instead.  The
+// 16-byte response lands in shared memory at `resp` (16-byte aligned) and
+// completes 16 transaction bytes on `bar`.  Issued by one elected lane; after a
+// response that reports failure no further request may be made.
+__device__ __forceinline__ void clc_try_cancel_elect(uint32_t resp, uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%1], 16;\n\t"
+        "@e clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];\n\t"
+        "}" ::"r"(resp),
+        "r"(bar)
+        : "memory");
+}
+
+// Decodes a response: the x index of the cancelled CTA, or -1 when nothing
+// was cancelled (every CTA of the grid has started or been taken).
+__device__ __forceinline__ int clc_query_x(uint32_t resp) {
+    int x;
+    asm volatile(
+        "{\n\t.reg .b128 r;\n\t.reg .pred ok;\n\t.reg .b32 cx;\n\t"
+        "ld.shared.b128 r, [%1];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 ok, r;\n\t"
+        "mov.b32 cx, -1;\n\t"
+        "@ok clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 cx, r;\n\t"
+        "mov.b32 %0, cx;\n\t"
+        "}"
+        : "=r"(x)
+        : "r"(resp)
+        : "memory");
+    return x;
+}
+
 }  // namespace ptx
 }  // namespace attn
