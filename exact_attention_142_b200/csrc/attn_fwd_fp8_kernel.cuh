@@ -98,9 +98,13 @@ struct Layout {
     static constexpr uint32_t kQ1 = kTileBytes;
     static constexpr uint32_t kKV = 2 * kTileBytes;
     static constexpr uint32_t kBar = kKV + kStages * kTileBytes;
-    static constexpr uint32_t kNumBars = 8 + 2 * kStages;
-    static constexpr uint32_t kMisc = kBar + kNumBars * 8;
-    static constexpr uint32_t kBytes = kMisc + 16;
+    // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
+    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2]
+    static constexpr uint32_t kNumBars = 16 + 2 * kStages;
+    static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem address, abort flag
+    static constexpr uint32_t kClcResp = kMisc + 16;        // launch-control response (16 B)
+    static constexpr uint32_t kUnitQ = kClcResp + 16;       // unit queue: two ints
+    static constexpr uint32_t kBytes = kUnitQ + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 
     static __device__ __forceinline__ uint32_t bar_q(uint32_t base) { return base + kBar; }
@@ -120,6 +124,21 @@ struct Layout {
     static __device__ __forceinline__ uint32_t bar_mma_final(uint32_t base) {
         return base + kBar + 8u * (7 + 2 * kStages);
     }
+    static __device__ __forceinline__ uint32_t bar_q_empty(uint32_t base) {
+        return base + kBar + 8u * (8 + 2 * kStages);
+    }
+    static __device__ __forceinline__ uint32_t bar_o_free(uint32_t base, int x) {
+        return base + kBar + 8u * (9 + 2 * kStages + x);
+    }
+    static __device__ __forceinline__ uint32_t bar_clc(uint32_t base) {
+        return base + kBar + 8u * (11 + 2 * kStages);
+    }
+    static __device__ __forceinline__ uint32_t bar_unit_full(uint32_t base, int slot) {
+        return base + kBar + 8u * (12 + 2 * kStages + slot);
+    }
+    static __device__ __forceinline__ uint32_t bar_unit_empty(uint32_t base, int slot) {
+        return base + kBar + 8u * (14 + 2 * kStages + slot);
+    }
 };
 
 // First padded column of sequence b in V^T (each sequence rounded up to 128).
@@ -130,41 +149,50 @@ __device__ __forceinline__ int vt_start(const FwdParams& p, int b) {
     return s;
 }
 
-__device__ __forceinline__ void producer(const TilePair& w, const FwdParams& p, const CUtensorMap* tm_q,
-                                         const CUtensorMap* tm_k, const CUtensorMap* tm_vt, uint32_t sbase,
-                                         volatile int* abort_flag) {
+// The bf16 kernel's persistent schedule (UnitSource), with V^T blocks.
+__device__ __forceinline__ void producer(const FwdParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                         const CUtensorMap* tm_vt, uint32_t sbase, volatile int* abort_flag) {
     using L = Layout;
+    const unsigned long long lim = p.wait_limit_ns;
     const uint64_t pol_q = ptx::policy_evict_first();
     const uint64_t pol_kv = ptx::policy_evict_last();
-    const int vs = vt_start(p, w.b);
-    ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * kTileBytes);
-    for (int x = 0; x < 2; ++x)
-        ptx::tma_load_2d_elect(sbase + (x ? L::kQ1 : L::kQ0), tm_q, L::bar_q(sbase), w.h[x] * kD,
-                               w.start + w.r0[x], pol_q);
-    int issued = 0;
+    UnitSource<L> src(sbase);
+    int issued = 0;  // K/V ring loads
+    int units = 0;   // pairs whose Q was loaded
     bool ok = true;
-    for (int j = w.ulo; j < w.uhi && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv) {
-            const int s = issued % kStages;
-            const uint32_t ph = (issued / kStages) & 1;
-            if (!warp_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, p.wait_limit_ns)) {
-                ok = false;
-                break;
+    int u = src.next(p, abort_flag, ok);
+    while (ok) {
+        if (!(ok = src.publish(u, abort_flag, lim)) || u < 0) break;
+        const TilePair w = decode_pair(u, p);
+        const int vs = vt_start(p, w.b);
+        if (units > 0 && !(ok = warp_wait(L::bar_q_empty(sbase), (units - 1) & 1, abort_flag, lim))) break;
+        ptx::mbar_arrive_expect_tx_elect(L::bar_q(sbase), 2 * kTileBytes);
+        for (int x = 0; x < 2; ++x)
+            ptx::tma_load_2d_elect(sbase + (x ? L::kQ1 : L::kQ0), tm_q, L::bar_q(sbase), w.h[x] * kD,
+                                   w.start + w.r0[x], pol_q);
+        ++units;
+        for (int j = w.ulo; j < w.uhi && ok; ++j) {
+            for (int kv = 0; kv < 2; ++kv) {
+                const int s = issued % kStages;
+                const uint32_t ph = (issued / kStages) & 1;
+                if (!(ok = warp_wait(L::bar_kv_empty(sbase, s), ph ^ 1, abort_flag, lim))) break;
+                ptx::mbar_arrive_expect_tx_elect(L::bar_kv_full(sbase, s), kTileBytes);
+                if (kv == 0)  // K block: 128 keys x 128 values of head g
+                    ptx::tma_load_2d_elect(sbase + L::kKV + s * kTileBytes, tm_k, L::bar_kv_full(sbase, s),
+                                           w.g * kD, w.start + j * kBN, pol_kv);
+                else  // V^T block: 128 values of head g x 128 keys
+                    ptx::tma_load_2d_elect(sbase + L::kKV + s * kTileBytes, tm_vt, L::bar_kv_full(sbase, s),
+                                           vs + j * kBN, w.g * kD, pol_kv);
+                ++issued;
             }
-            ptx::mbar_arrive_expect_tx_elect(L::bar_kv_full(sbase, s), kTileBytes);
-            if (kv == 0)  // K block: 128 keys x 128 values of head g
-                ptx::tma_load_2d_elect(sbase + L::kKV + s * kTileBytes, tm_k, L::bar_kv_full(sbase, s),
-                                       w.g * kD, w.start + j * kBN, pol_kv);
-            else  // V^T block: 128 values of head g x 128 keys
-                ptx::tma_load_2d_elect(sbase + L::kKV + s * kTileBytes, tm_vt, L::bar_kv_full(sbase, s),
-                                       vs + j * kBN, w.g * kD, pol_kv);
-            ++issued;
         }
+        if (ok) u = src.next(p, abort_flag, ok);
     }
-    drain_wait(L::bar_q(sbase), 0, p.wait_limit_ns);
+    src.drain(lim);
+    if (units > 0) drain_wait(L::bar_q(sbase), (units - 1) & 1, lim);
     const int first = issued > kStages ? issued - kStages : 0;
     for (int i = first; i < issued; ++i)
-        drain_wait(L::bar_kv_full(sbase, i % kStages), (i / kStages) & 1, p.wait_limit_ns);
+        drain_wait(L::bar_kv_full(sbase, i % kStages), (i / kStages) & 1, lim);
 }
 
 __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, int slot) {
@@ -189,80 +217,24 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
                         ptx::smem_desc_sw128(va + kk * 32, 16, 1024), kIdesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// The bf16 kernel's MMA order and barriers (S0(j), PV1(j-1), S1(j), PV0(j)).
-__device__ __forceinline__ void mma_role(const TilePair& w, const FwdParams& p, uint32_t tmem, uint32_t sbase,
+// The bf16 kernel's MMA loop (order S0(j), PV1(j-1), S1(j), PV0(j), and its
+// barriers) with the e4m3 products.
+__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint32_t sbase,
                                          volatile int* abort_flag) {
-    using L = Layout;
-    const unsigned long long lim = p.wait_limit_ns;
-    bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
-    ptx::tc_fence_after_sync();
-    int pc[2] = {0, 0};
-    bool first[2] = {true, true};
-    for (int j = w.ulo; ok && j < w.uhi; ++j) {
-        const int kidx = 2 * (j - w.ulo), vidx = kidx + 1;
-        const int ks = kidx % kStages, vs = vidx % kStages;
-        if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (kidx / kStages) & 1, abort_flag, lim))) break;
-        ptx::tc_fence_after_sync();
-        if (tile_active_at(w, 0, j)) {
-            issue_qk(tmem, sbase, 0, ks);
-            ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
-        }
-        if (j > w.ulo) {
-            const int pvs = (vidx - 2) % kStages;
-            if (tile_active_at(w, 1, j - 1)) {
-                if (!(ok = warp_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim))) break;
-                ++pc[1];
-                ptx::tc_fence_after_sync();
-                issue_pv(tmem, sbase, 1, pvs, !first[1]);
-                first[1] = false;
-                if (j - 1 == w.hi[1] - 1) ptx::tc_commit_elect(L::bar_o_done(sbase, 1));
-            }
-            ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
-        }
-        if (tile_active_at(w, 1, j)) {
-            issue_qk(tmem, sbase, 1, ks);
-            ptx::tc_commit_elect(L::bar_s_full(sbase, 1));
-        }
-        ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
-        if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), (vidx / kStages) & 1, abort_flag, lim))) break;
-        ptx::tc_fence_after_sync();
-        if (tile_active_at(w, 0, j)) {
-            if (!(ok = warp_wait(L::bar_p_ready(sbase, 0), pc[0] & 1, abort_flag, lim))) break;
-            ++pc[0];
-            ptx::tc_fence_after_sync();
-            issue_pv(tmem, sbase, 0, vs, !first[0]);
-            first[0] = false;
-            if (j == w.hi[0] - 1) ptx::tc_commit_elect(L::bar_o_done(sbase, 0));
-        }
-    }
-    if (ok && w.uhi > w.ulo) {
-        const int j = w.uhi - 1;
-        const int vs = (2 * (j - w.ulo) + 1) % kStages;
-        if (tile_active_at(w, 1, j)) {
-            ok = warp_wait(L::bar_p_ready(sbase, 1), pc[1] & 1, abort_flag, lim);
-            if (ok) {
-                ptx::tc_fence_after_sync();
-                issue_pv(tmem, sbase, 1, vs, !first[1]);
-                ptx::tc_commit_elect(L::bar_o_done(sbase, 1));
-            }
-        }
-        ptx::tc_commit_elect(L::bar_kv_empty(sbase, vs));
-    }
-    ptx::tc_commit_elect(L::bar_mma_final(sbase));
-    drain_wait(L::bar_mma_final(sbase), 0, lim);
+    mma_loop<Layout, kStages>(
+        p, sbase, abort_flag, [&](int x, int slot) { issue_qk(tmem, sbase, x, slot); },
+        [&](int x, int slot, bool acc) { issue_pv(tmem, sbase, x, slot, acc); });
 }
 
 // One thread per query row, as in the bf16 kernel; P goes to tensor memory as
 // e4m3 (4 per column).
-__device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams& p, int x, int warp_in_group,
-                                             int lane, uint32_t tmem, uint32_t sbase, volatile int* abort_flag) {
+__device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams& p, int x, int warp_in_group,
+                                             int lane, uint32_t tmem, uint32_t sbase, volatile int* abort_flag,
+                                             uint32_t& phases, int u) {
     using L = Layout;
-    const bool active = x ? w.active[1] : w.active[0];
-    if (!active) return;
     const int r0 = x ? w.r0[1] : w.r0[0];
     const int blk_lo = x ? w.lo[1] : w.lo[0];
     const int blk_hi = x ? w.hi[1] : w.hi[0];
-    const int h = x ? w.h[1] : w.h[0];
     const unsigned long long lim = p.wait_limit_ns;
     const int row = r0 + warp_in_group * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
@@ -281,8 +253,9 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
     float l_q = 0.0f;    // e4m3-rounded weights -> O
     bool ok = true;
     for (int j = blk_lo; j < blk_hi; ++j) {
-        ok = __all_sync(0xffffffffu, bounded_wait(L::bar_s_full(sbase, x), (j - blk_lo) & 1, abort_flag, lim));
+        ok = __all_sync(0xffffffffu, bounded_wait(L::bar_s_full(sbase, x), phases & 1u, abort_flag, lim));
         if (!ok) break;
+        phases ^= 1u;
         ptx::tc_fence_after_sync();
         uint32_t s[128];
         ptx::tmem_ld128_sync(t_s, s);
@@ -372,13 +345,18 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
         ptx::tc_fence_before_sync();
         ptx::mbar_arrive(L::bar_p_ready(sbase, x));
     }
-    if (!ok) return;
-    ok = __all_sync(0xffffffffu, bounded_wait(L::bar_o_done(sbase, x), 0, abort_flag, lim));
-    if (!ok) return;
+    if (!ok) return false;
+    ok = __all_sync(0xffffffffu, bounded_wait(L::bar_o_done(sbase, x), (phases >> 1) & 1u, abort_flag, lim));
+    if (!ok) return false;
     ptx::tc_fence_after_sync();
-    const bool store = row < w.len;
+    // The pair's indices again (recomputed rather than kept live through the loop).
+    int u_again = u;
+    asm volatile("" : "+r"(u_again));
+    const TilePair we = decode_pair(u_again, p);
+    const int h = x ? we.h[1] : we.h[0];
+    const bool store = row < we.len;
     const float inv = l_q > 0.0f ? 1.0f / l_q : 0.0f;
-    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)(w.start + (store ? row : 0)) * p.Hq + h) * (size_t)kD * 2;
+    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)(we.start + (store ? row : 0)) * p.Hq + h) * (size_t)kD * 2;
 #pragma unroll
     for (int cc = 0; cc < kD / 32; ++cc) {
         uint32_t o[32];
@@ -395,8 +373,28 @@ __device__ __forceinline__ void softmax_role(const TilePair& w, const FwdParams&
     }
     if (store) {
         const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
-        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + w.start + row : ((size_t)w.b * p.Hq + h) * p.N + row;
+        const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + row : ((size_t)we.b * p.Hq + h) * p.N + row;
         p.lse[idx] = lse;
+    }
+    // O has been read: the next pair's first PV of this tile may overwrite it
+    ptx::tc_fence_before_sync();
+    ptx::mbar_arrive(L::bar_o_free(sbase, x));
+    return true;
+}
+
+// The pairs of this CTA for one tile (tiles with no rows skipped).
+__device__ __forceinline__ void softmax_role(const FwdParams& p, int x, int warp_in_group, int lane, uint32_t tmem,
+                                             uint32_t sbase, volatile int* abort_flag) {
+    // bit 0: s_full parity, bit 1: o_done parity, bits 2-3: unit queue index mod 4
+    uint32_t phases = 0;
+    while (true) {
+        const int u = unit_take<Layout>(sbase, phases >> 2, abort_flag, p.wait_limit_ns);
+        phases = (phases + 4u) & 15u;
+        if (u < 0) break;
+        const TilePair w = decode_pair(u, p);
+        if (!(x ? w.active[1] : w.active[0])) continue;
+        if (!softmax_unit(w, p, x, warp_in_group, lane, tmem, sbase, abort_flag, phases, u)) return;
+        phases ^= 2u;
     }
 }
 
@@ -410,8 +408,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = ptx::smem_addr(smem);
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const TilePair w = decode_pair(blockIdx.x, p);
-    if (!w.active[0] && !w.active[1]) return;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     if (warp == kWarpProducer && lane == 0) {
@@ -426,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(L::bar_o_done(sbase, x), 1);
         }
         ptx::mbar_init(L::bar_mma_final(sbase), 1);
+        init_schedule_barriers<L>(sbase);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_q);
@@ -442,13 +439,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     if (warp < 8) {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
-        softmax_role(w, p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
+        softmax_role(p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (warp == kWarpProducer)
-            producer(w, p, &tm_q, &tm_k, &tm_vt, sbase, abort_flag);
+            producer(p, &tm_q, &tm_k, &tm_vt, sbase, abort_flag);
         else if (warp == kWarpMma)
-            mma_role(w, p, tmem, sbase, abort_flag);
+            mma_role(p, tmem, sbase, abort_flag);
     }
     ptx::tc_fence_before_sync();
     __syncthreads();

@@ -287,7 +287,7 @@ __device__ __forceinline__ bool tile_active_at(const TilePair& w, int x, int j) 
     return w.active[x] && j >= w.lo[x] && j < w.hi[x];
 }
 
-// ---------------------------------------------------------------- producer
+// ---------------------------------------------------------------- schedule
 // Persistent, varlen-aware schedule.  The grid holds one CTA per tile pair in
 // heaviest-first order.  A running CTA starts with its own pair; when the
 // producer has issued every load of a pair it takes the next pending pair by
@@ -297,27 +297,25 @@ __device__ __forceinline__ bool tile_active_at(const TilePair& w, int x, int j) 
 // queue in shared memory.  Pairs are thus handed out greedily in the same
 // order as by the hardware's block scheduler, while the next pair's Q load
 // and first products overlap the previous pair's epilogue.
-template <int D, int STAGES>
-__device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensorMap* tm_q,
-                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                              uint32_t sbase, volatile int* abort_flag) {
-    using L = SmemLayout<D, STAGES>;
-    constexpr int kBoxes = D / 64;
-    const unsigned long long lim = p.wait_limit_ns;
-    const uint64_t pol_q = ptx::policy_evict_first();
-    const uint64_t pol_kv = ptx::policy_evict_last();
-    const uint32_t resp = sbase + L::kClcResp;
-    int issued = 0;      // K/V ring loads
-    int units = 0;       // pairs whose Q was loaded
-    int published = 0;   // unit queue entries written
-    int requests = 0;    // launch-control requests answered
-    bool pending = false;  // a request whose answer has not been seen
-    bool more = true;      // false after a request that cancelled nothing
-    int cand = blockIdx.x;
-    bool ok = true;
+//
+// UnitSource is the producer warp's side.  L provides bar_clc, kClcResp,
+// kUnitQ, bar_unit_full and bar_unit_empty.
+template <class L>
+struct UnitSource {
+    uint32_t sbase;
+    int cand;          // next pair to examine (-1: ask the hardware)
+    int requests;      // launch-control requests answered
+    int published;     // unit queue entries written
+    bool pending;      // a request whose answer has not been seen
+    bool more;         // false after a request that cancelled nothing
 
-    // The next pair with rows, or -1.
-    auto next_unit = [&]() -> int {
+    __device__ __forceinline__ explicit UnitSource(uint32_t base)
+        : sbase(base), cand(blockIdx.x), requests(0), published(0), pending(false), more(true) {}
+
+    // The next pair with rows, or -1 (the grid is exhausted, or a wait timed
+    // out: then ok is cleared).  Called by the whole warp.
+    __device__ __forceinline__ int next(const FwdParams& p, volatile int* abort_flag, bool& ok) {
+        const uint32_t resp = sbase + L::kClcResp;
         while (true) {
             if (cand >= 0) {
                 const TilePair w = decode_pair(cand, p);
@@ -330,7 +328,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensor
             __syncwarp();
             ptx::clc_try_cancel_elect(resp, L::bar_clc(sbase));
             pending = true;
-            if (!warp_wait(L::bar_clc(sbase), requests & 1, abort_flag, lim)) {
+            if (!warp_wait(L::bar_clc(sbase), requests & 1, abort_flag, p.wait_limit_ns)) {
                 ok = false;
                 return -1;
             }
@@ -339,8 +337,10 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensor
             cand = ptx::clc_query_x(resp);
             if (cand < 0) more = false;
         }
-    };
-    auto publish = [&](int u) -> bool {
+    }
+
+    // Hands pair u (or -1: no more work) to the MMA and softmax warps.
+    __device__ __forceinline__ bool publish(int u, volatile int* abort_flag, unsigned long long lim) {
         const int slot = published & 1;
         if (!warp_wait(L::bar_unit_empty(sbase, slot), ((published >> 1) & 1) ^ 1, abort_flag, lim))
             return false;
@@ -349,11 +349,43 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensor
         if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(L::bar_unit_full(sbase, slot));
         ++published;
         return true;
-    };
+    }
 
-    int u = next_unit();
+    // A request still in flight must land before the block exits.
+    __device__ __forceinline__ void drain(unsigned long long lim) {
+        if (pending) drain_wait(L::bar_clc(sbase), requests & 1, lim);
+    }
+};
+
+// Initialises the schedule's barriers (one thread).
+template <class L>
+__device__ __forceinline__ void init_schedule_barriers(uint32_t sbase) {
+    ptx::mbar_init(L::bar_q_empty(sbase), 1);
+    for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_o_free(sbase, x), 128);
+    ptx::mbar_init(L::bar_clc(sbase), 1);
+    for (int slot = 0; slot < 2; ++slot) {
+        ptx::mbar_init(L::bar_unit_full(sbase, slot), 1);
+        ptx::mbar_init(L::bar_unit_empty(sbase, slot), kUnitReaders);
+    }
+}
+
+// ---------------------------------------------------------------- producer
+template <int D, int STAGES>
+__device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              uint32_t sbase, volatile int* abort_flag) {
+    using L = SmemLayout<D, STAGES>;
+    constexpr int kBoxes = D / 64;
+    const unsigned long long lim = p.wait_limit_ns;
+    const uint64_t pol_q = ptx::policy_evict_first();
+    const uint64_t pol_kv = ptx::policy_evict_last();
+    UnitSource<L> src(sbase);
+    int issued = 0;  // K/V ring loads
+    int units = 0;   // pairs whose Q was loaded
+    bool ok = true;
+    int u = src.next(p, abort_flag, ok);
     while (ok) {
-        if (!(ok = publish(u)) || u < 0) break;
+        if (!(ok = src.publish(u, abort_flag, lim)) || u < 0) break;
         const TilePair w = decode_pair(u, p);
         // the previous pair's score products have finished reading Q
         if (units > 0 && !(ok = warp_wait(L::bar_q_empty(sbase), (units - 1) & 1, abort_flag, lim))) break;
@@ -378,10 +410,10 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensor
                 ++issued;
             }
         }
-        if (ok) u = next_unit();
+        if (ok) u = src.next(p, abort_flag, ok);
     }
     // Every copy and request issued must have landed before the block may exit.
-    if (pending) drain_wait(L::bar_clc(sbase), requests & 1, lim);
+    src.drain(lim);
     if (units > 0) drain_wait(L::bar_q(sbase), (units - 1) & 1, lim);
     const int first = issued > STAGES ? issued - STAGES : 0;
     for (int i = first; i < issued; ++i) drain_wait(L::bar_kv_full(sbase, i % STAGES), (i / STAGES) & 1, lim);
@@ -423,10 +455,12 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
     }
 }
 
-template <int D, int STAGES>
-__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint32_t sbase,
-                                         volatile int* abort_flag) {
-    using L = SmemLayout<D, STAGES>;
+// The MMA warp's loop over the pairs of its CTA.  qk(x, slot) issues the score
+// product of tile x from ring slot `slot`; issue(x, slot, accumulate) the P V
+// product.  Shared by the bf16 and the e4m3 kernels.
+template <class L, int STAGES, class IssueQK, class IssuePV>
+__device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, volatile int* abort_flag,
+                                         IssueQK&& qk, IssuePV&& issue) {
     const unsigned long long lim = p.wait_limit_ns;
     // Phase bits, kept in one word (this warp runs with few registers):
     enum : uint32_t {
@@ -453,7 +487,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
         return true;
     };
     auto pv = [&](int x, int slot, bool last) {
-        issue_pv<D, STAGES>(tmem, sbase, x, slot, !(f & (kFirst << x)));
+        issue(x, slot, !(f & (kFirst << x)));
         f &= ~(kFirst << x);
         if (last) {
             ptx::tc_commit_elect(L::bar_o_done(sbase, x));
@@ -479,7 +513,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
             if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (ring / STAGES) & 1, abort_flag, lim))) break;
             ptx::tc_fence_after_sync();
             if (j >= lo0 && j < hi0) {
-                issue_qk<D, STAGES>(tmem, sbase, 0, ks);
+                qk(0, ks);
                 ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
             }
             if (j > w.ulo) {
@@ -491,7 +525,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
                 ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
             }
             if (j >= lo1 && j < hi1) {
-                issue_qk<D, STAGES>(tmem, sbase, 1, ks);
+                qk(1, ks);
                 ptx::tc_commit_elect(L::bar_s_full(sbase, 1));
             }
             ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
@@ -519,6 +553,14 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
     // All MMAs must be complete before tensor memory is released.
     ptx::tc_commit_elect(L::bar_mma_final(sbase));
     drain_wait(L::bar_mma_final(sbase), 0, lim);
+}
+
+template <int D, int STAGES>
+__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint32_t sbase,
+                                         volatile int* abort_flag) {
+    mma_loop<SmemLayout<D, STAGES>, STAGES>(
+        p, sbase, abort_flag, [&](int x, int slot) { issue_qk<D, STAGES>(tmem, sbase, x, slot); },
+        [&](int x, int slot, bool acc) { issue_pv<D, STAGES>(tmem, sbase, x, slot, acc); });
 }
 
 // ---------------------------------------------------------------- softmax
@@ -788,13 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(L::bar_o_done(sbase, x), 1);
         }
         ptx::mbar_init(L::bar_mma_final(sbase), 1);
-        ptx::mbar_init(L::bar_q_empty(sbase), 1);
-        for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_o_free(sbase, x), 128);
-        ptx::mbar_init(L::bar_clc(sbase), 1);
-        for (int slot = 0; slot < 2; ++slot) {
-            ptx::mbar_init(L::bar_unit_full(sbase, slot), 1);
-            ptx::mbar_init(L::bar_unit_empty(sbase, slot), kUnitReaders);
-        }
+        init_schedule_barriers<L>(sbase);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_q);
