@@ -563,11 +563,16 @@ struct DqLayout {
     static constexpr uint32_t kRing = 2 * kTileQ;
     static constexpr uint32_t kSlot = 2 * kTileK;  // K, V
     static constexpr uint32_t kBar = kRing + STAGES * kSlot;
-    // q_loaded, slot_full[S], slot_empty[S], st_full[2], ds_ready[2], done
-    static constexpr uint32_t kNumBars = 6 + 2 * STAGES;
+    // q_loaded, slot_full[S], slot_empty[S], st_full[2], ds_ready[2], done, a_ready
+    static constexpr uint32_t kNumBars = 7 + 2 * STAGES;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
+    // Tensor memory: S [0,128) and dP [128,256) as two 64-column buffers each,
+    // dQ [256, 256 + D), then Q and dO as bf16 pairs (D / 2 columns each): the
+    // A operands of the S and dP products.
+    static constexpr uint32_t kTQ = 384;
+    static constexpr uint32_t kTDO = kTQ + D / 2;
 
     static __device__ __forceinline__ uint32_t k(uint32_t base, int s) { return base + kRing + s * kSlot; }
     static __device__ __forceinline__ uint32_t v(uint32_t base, int s) { return k(base, s) + kTileK; }
@@ -583,7 +588,39 @@ struct DqLayout {
         return base + kBar + 8u * (3 + 2 * STAGES + b);
     }
     static __device__ __forceinline__ uint32_t bar_done(uint32_t base) { return base + kBar + 8u * (5 + 2 * STAGES); }
+    static __device__ __forceinline__ uint32_t bar_a(uint32_t base) { return base + kBar + 8u * (6 + 2 * STAGES); }
 };
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// Copies this thread's row of Q (groups 0, 1) or dO (groups 2, 3) from the
+// TMA tile (128-byte swizzle: 16-byte chunk c of row r sits at chunk
+// c ^ (r mod 8) of its 128-byte line) into tensor memory, half a row per
+// group, packed two bf16 per column in the order of d.
+template <int D, int STAGES>
+__device__ __forceinline__ void dq_stage_a(uint32_t tl, uint32_t sbase, int x, int row) {
+    using L = DqLayout<D, STAGES>;
+    constexpr int kChunks = D / 16;  // 16-byte chunks in half a row
+    const uint32_t src = sbase + (x < 2 ? L::kQ : L::kDO);
+    const int c0 = (x & 1) * kChunks;
+    uint32_t r[4 * kChunks];
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int c = c0 + i;
+        const uint32_t addr = src + (c >> 3) * kBox128 + row * 128 + (((c & 7) ^ (row & 7)) << 4);
+        ld_shared_v4(addr, r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+    }
+    const uint32_t dst = tl + (x < 2 ? L::kTQ : L::kTDO) + 4 * c0;
+    if constexpr (kChunks == 8)
+        ptx::tmem_st32(dst, r);
+    else
+        ptx::tmem_st16(dst, r);
+}
 
 struct DqWork {
     int b, h, g, m, start, len, n_lo, n_hi;
@@ -652,21 +689,25 @@ __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint
     constexpr uint32_t kIdG = ptx::idesc_bf16_f32(kBM, D, false, true);
     const unsigned long long lim = p.wait_limit_ns;
     const int steps = w.n_hi - w.n_lo;
-    bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
+    // Q and dO reach tensor memory through the elementwise warps (dq_stage_a).
+    bool ok = warp_wait(L::bar_a(sbase), 0, abort_flag, lim);
     ptx::tc_fence_after_sync();
     auto issue_st = [&](int t) -> bool {  // S(t) and dP(t) into buffer t & 1
         const int s = t % STAGES;
         if (!warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim)) return false;
         ptx::tc_fence_after_sync();
         const uint32_t buf = (t & 1) * 64;
+        // A from tensor memory: shared memory then serves only the 64-key B
+        // operand (an SS product of N = 64 would read 1.5x the shared-memory
+        // bandwidth that the tensor pipe consumes).
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)  // S = Q K^T
-            ptx::mma_ss_elect(tmem + buf, kmajor_desc(sbase + L::kQ, kk, kBox128),
-                              kmajor_desc(L::k(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
+            ptx::mma_ts_elect(tmem + buf, tmem + L::kTQ + 8 * kk, kmajor_desc(L::k(sbase, s), kk, kBox64), kIdS,
+                              kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)  // dP = dO V^T
-            ptx::mma_ss_elect(tmem + 128 + buf, kmajor_desc(sbase + L::kDO, kk, kBox128),
-                              kmajor_desc(L::v(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
+            ptx::mma_ts_elect(tmem + 128 + buf, tmem + L::kTDO + 8 * kk, kmajor_desc(L::v(sbase, s), kk, kBox64),
+                              kIdS, kk > 0 ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_st(sbase, t & 1));
         return true;
     };
@@ -708,8 +749,14 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
         dd = p.dsum[idx];
     }
     const unsigned long long lim = p.wait_limit_ns;
-    bool ok = true;
-    for (int n = w.n_lo; n < w.n_hi; ++n) {
+    bool ok = warp_wait(L::bar_q(sbase), 0, abort_flag, lim);
+    if (ok) {
+        dq_stage_a<D, STAGES>(tl, sbase, x, row);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before_sync();
+        ptx::mbar_arrive(L::bar_a(sbase));
+    }
+    for (int n = w.n_lo; ok && n < w.n_hi; ++n) {
         const int t = n - w.n_lo;
         const uint32_t buf = (t & 1) * 64;
         if (!(ok = warp_wait(L::bar_st(sbase, t & 1), (t >> 1) & 1, abort_flag, lim))) break;
@@ -787,6 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(L::bar_ds(sbase, b), kElemThreads);
         }
         ptx::mbar_init(L::bar_done(sbase), 1);
+        ptx::mbar_init(L::bar_a(sbase), kElemThreads);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_q);
