@@ -249,3 +249,63 @@ def test_empty_inputs_enqueue_nothing():
 def test_wrong_device_arch_is_not_silently_used():
     major, minor = torch.cuda.get_device_capability()
     assert (major, minor) == (10, 0), "these kernels are built for sm_100a only"
+
+
+# The persistent schedule: one CTA per SM takes over the tile pairs of CTAs that
+# have not started, so most CTAs compute many pairs in a row; per-pair state
+# (running maximum and sums, barrier phases, the O hand-over between a pair's
+# epilogue and the next pair's first P V) must not leak between pairs.  Pairs
+# past a packed sequence's end are skipped by the producer.
+SCHEDULE_CASES = [
+    # (name, B, Hq, Hkv, N, d, causal, left, right, seed): a few hundred pairs each
+    ("heads_paired_causal", 32, 8, 2, 300, 128, True, -1, -1, 31),
+    ("rows_paired_noncausal_d64", 24, 6, 6, 520, 64, False, -1, -1, 32),
+    ("heads_paired_window_d64", 16, 8, 4, 700, 64, True, 90, 0, 33),
+]
+
+
+@pytest.mark.parametrize("case", SCHEDULE_CASES, ids=lambda c: c[0])
+def test_schedule_many_pairs_per_cta(case):
+    name, B, Hq, Hkv, N, d, causal, left, right, seed = case
+    q, k, v = W.draw_qkv((B, N, Hq, d), (B, N, Hkv, d), seed)
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=causal,
+              window_left=left, window_right=right)
+    o, lse = gpu_run(q, k, v, **kw)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    compare_full(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_schedule_mostly_empty_packed(d):
+    """Most tile pairs lie past their sequence's end (many empty and one-token
+    sequences beside a long one); every row is still computed, once."""
+    lengths = [0] * 40 + [1] * 20 + [700] + [0] * 30 + [129, 2, 0, 255]
+    cu = W.cumulative(lengths)
+    T, Hq, Hkv = cu[-1], 4, 2
+    q, k, v = W.draw_qkv((T, Hq, d), (T, Hkv, d), 40 + d)
+    kw = dict(B=len(lengths), Hq=Hq, Hkv=Hkv, N=T, d=d, scale=default_scale(d), causal=True,
+              cu_seqlens=cu)
+    o, lse = gpu_run(q, k, v, **kw)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    compare_full(o, lse, o_ref, lse_ref)
+
+
+def test_schedule_accumulate_many_pairs():
+    """The accumulating epilogue under the persistent schedule: one call into an
+    empty accumulator (O = 0, LSE = -inf) gives the attention output itself."""
+    B, Hq, Hkv, N, d = 24, 8, 2, 384, 128
+    q, k, v = W.draw_qkv((B, N, Hq, d), (B, N, Hkv, d), 34)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o_acc = torch.zeros((B, N, Hq, d), dtype=torch.float32, device=dev)
+    l_acc = torch.full((B, Hq, N), float("-inf"), dtype=torch.float32, device=dev)
+    scale = default_scale(d)
+    assert ea.attn_fwd_accumulate(qd, kd, vd, o_acc, l_acc, B, Hq, Hkv, N, d, scale,
+                                  True) == ea.ATTN_OK
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    o_ref, lse_ref, _ = oracle_run(q, k, v, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=scale,
+                                   causal=True)
+    # fp32 output: only the weights' bf16 rounding remains (no output rounding)
+    assert float(np.abs(o_acc.cpu().double().numpy() - o_ref.reshape(B, N, Hq, d)).max()) <= 5e-3
+    assert float(np.abs(l_acc.cpu().double().numpy() - lse_ref.reshape(B, Hq, N)).max()) <= TOL_LSE

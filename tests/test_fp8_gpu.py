@@ -197,3 +197,30 @@ def test_fp8_gqa_workload_sampled_rows():
     rows = [(b, h, i, r, b * N + i) for r, (b, h, i) in enumerate(picks)]
     check_rows(og, np.array([lg[b, h, i] for b, h, i in picks]), o_ref, lse_ref, qf, kf, vf, rows,
                scale, True, -1, -1, [N] * B, Hq // Hkv)
+
+
+def test_fp8_schedule_many_pairs_per_cta():
+    """Several hundred tile pairs (many per CTA under the persistent schedule),
+    ragged tail, GQA."""
+    B, Hq, Hkv, N, d = 16, 8, 2, 300, 128
+    q, k, v = W.draw_qkv_e4m3((B, N, Hq, d), (B, N, Hkv, d), seed=35)
+    scale = default_scale(d)
+    o_gpu, lse_gpu = gpu_fp8(q, k, v, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=scale, causal=True)
+    o_ref, lse_ref, _ = oracle_fp8(q, k, v, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=scale, causal=True)
+    T = B * N
+    qf = W.e4m3_as_bf16(q).double().numpy().reshape(T, Hq, d)
+    kf = W.e4m3_as_bf16(k).double().numpy().reshape(T, Hkv, d)
+    vf = W.e4m3_as_bf16(v).double().numpy().reshape(T, Hkv, d)
+    og = o_gpu.double().numpy().reshape(T, Hq, d)
+    lg = lse_gpu.double().numpy().reshape(B, Hq, N)
+    o_ref = o_ref.reshape(T, Hq, d)
+    rng = np.random.default_rng(36)
+    picks = [(b, h, i) for b in (0, B - 1) for h in (0, Hq - 1) for i in (0, 127, 128, 255, 256, N - 1)]
+    picks += [(int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(N))) for _ in range(200)]
+    rows = [(b, h, i, r, b * N + i) for r, (b, h, i) in enumerate(picks)]
+    check_rows(og, np.array([lg[b, h, i] for b, h, i in picks]),
+               np.array([o_ref[b * N + i, h] for b, h, i in picks]),
+               np.array([lse_ref[b, h, i] for b, h, i in picks]), qf, kf, vf, rows, scale, True,
+               -1, -1, [N] * B, Hq // Hkv)
+    # every row of every pair was written
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
