@@ -297,6 +297,7 @@ def run_cuda(args, w: W.Workload, rank: int, world: int, local_rank: int):
         t = torch.tensor([kernel_ms, e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         kernel_ms, e2e_ms = float(t[0]), float(t[1])
+    run_cuda.step_times = sorted(times)
     return kernel_ms, e2e_ms, h2d, d2h, clocks
 
 
@@ -570,11 +571,81 @@ def calibrate_rows(w, q, k, v, target_s: float) -> int:
     return max(16, int(rows * target_s / max(dt, 1e-6)))
 
 
+def run_torch_sdpa(args, w: W.Workload):
+    """Context line: PyTorch's scaled_dot_product_attention on the same dense
+    workload (inputs as [B, H, N, d] copies), each backend that accepts it,
+    timed like the CUDA arm.  Sliding windows and packed sequences have no
+    direct SDPA form, so those workloads are reported unavailable."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    base = {"metric": METRIC, "unit": UNIT, "impl": "torch_sdpa (context, not this library)",
+            "config": config_dict(w, 1), "n_gpus": 1}
+    if w.packed or w.window_left >= 0 or (not w.causal and w.window_right >= 0):
+        return base | {"unavailable": "no sliding-window or packed form in scaled_dot_product_attention"}
+    dev = torch.device("cuda", 0)
+    q, k, v = W.inputs(w)
+    qd, kd, vd = (t.to(dev).transpose(1, 2).contiguous() for t in (q, k, v))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    fl = flops_of(w)
+    results = {}
+    for name, be in [("flash", SDPBackend.FLASH_ATTENTION), ("cudnn", SDPBackend.CUDNN_ATTENTION),
+                     ("efficient", SDPBackend.EFFICIENT_ATTENTION)]:
+        try:
+            with sdpa_kernel([be]):
+                def call():
+                    return F.scaled_dot_product_attention(qd, kd, vd, is_causal=w.causal, scale=w.scale,
+                                                          enable_gqa=w.Hq != w.Hkv)
+                for _ in range(args.warmup):
+                    call()
+                torch.cuda.synchronize(dev)
+                times = []
+                for _ in range(min(args.steps, 20)):
+                    flush.zero_()
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    call()
+                    b.record()
+                    torch.cuda.synchronize(dev)
+                    times.append(a.elapsed_time(b))
+            ms = sum(times) / len(times)
+            results[name] = {"ms": ms, "value": fl / (ms * 1e-3) / 1e12}
+        except RuntimeError as e:  # backend not available for this shape or device
+            results[name] = {"unavailable": str(e).splitlines()[0][:160]}
+    ok = [r["value"] for r in results.values() if "value" in r]
+    return base | {"value": max(ok) if ok else None, "backends": results,
+                   "higher_is_better": True, "dtype": "bf16"}
+
+
+def step_stats(times):
+    """Median and minimum of the timed steps (rank 0), beside the mean that
+    ms_per_step reports."""
+    if not times:
+        return None
+    t = sorted(times)
+    return {"mean": sum(t) / len(t), "median": t[len(t) // 2], "min": t[0], "max": t[-1],
+            "rank": 0}
+
+
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w: W.Workload, target_s: float = 12.0):
     q, k, v = W.inputs(w)
     rows = calibrate_rows(w, q, k, v, target_s)
     dt, fl, thr = oracle_sample(w, q, k, v, rows, seed=2)
     return {"value": fl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "cpu_model": host_cpu_model(),
             "sample": f"{rows} query rows drawn uniformly over (sequence, head, row) of the "
                       f"workload, fp64 oracle, {dt:.1f} s on {thr} threads"}
 
@@ -1117,7 +1188,9 @@ def main():
                     help="fwd: attn_fwd (the benchmark); bwd: attn_bwd on the same workload")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp8"],
                     help="fp8: the forward on e4m3 inputs (attn_fwd_fp8); d = 128 workloads")
-    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference", "torch_sdpa"],
+                    help="torch_sdpa: context only, PyTorch's scaled_dot_product_attention on the "
+                         "same dense workload (not this library; one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1143,6 +1216,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    if args.impl == "torch_sdpa":
+        if rank == 0:
+            print(json.dumps(run_torch_sdpa(args, w)), flush=True)
         return
 
     import torch
@@ -1180,6 +1257,7 @@ def main():
                          "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
                          "kernel": "attn_fwd_sm100<128,5>" if w.d == 128 else "attn_fwd_sm100<64,8>"},
             "clocks": clocks,
+            "step_ms": step_stats(run_cuda.step_times),
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
