@@ -120,8 +120,8 @@ struct SmemLayout {
     static constexpr uint32_t kKV = 2 * kTileBytes;
     static constexpr uint32_t kBar = kKV + STAGES * kTileBytes;
     // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
-    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2]
-    static constexpr uint32_t kNumBars = 16 + 2 * STAGES;
+    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_half[2]
+    static constexpr uint32_t kNumBars = 18 + 2 * STAGES;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem address, abort flag
     static constexpr uint32_t kClcResp = kMisc + 16;        // launch-control response (16 B)
     static constexpr uint32_t kUnitQ = kClcResp + 16;       // unit queue: two ints
@@ -161,6 +161,9 @@ struct SmemLayout {
     }
     static __device__ __forceinline__ uint32_t bar_unit_empty(uint32_t base, int slot) {
         return base + kBar + 8u * (14 + 2 * STAGES + slot);
+    }
+    static __device__ __forceinline__ uint32_t bar_p_half(uint32_t base, int x) {
+        return base + kBar + 8u * (16 + 2 * STAGES + x);
     }
 };
 
@@ -363,6 +366,7 @@ __device__ __forceinline__ void init_schedule_barriers(uint32_t sbase) {
     ptx::mbar_init(L::bar_q_empty(sbase), 1);
     for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_o_free(sbase, x), 128);
     ptx::mbar_init(L::bar_clc(sbase), 1);
+    for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_p_half(sbase, x), 128);
     for (int slot = 0; slot < 2; ++slot) {
         ptx::mbar_init(L::bar_unit_full(sbase, slot), 1);
         ptx::mbar_init(L::bar_unit_empty(sbase, slot), kUnitReaders);
@@ -437,8 +441,10 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, i
     }
 }
 
+// Keys [64 half, 64 half + 64) of the block: the softmax hands P over in two
+// halves, so the first half's product overlaps the second half's exponentials.
 template <int D, int STAGES>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot,
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot, int half,
                                          bool accumulate) {
     using L = SmemLayout<D, STAGES>;
     // B = V is [keys, d] with d contiguous: MN-major operand.  Swizzle atoms of
@@ -448,16 +454,18 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
     const uint32_t va = sbase + L::kKV + slot * L::kTileBytes;
     const uint32_t p_tmem = tmem + (x ? 128u : 0u) + kPOffset;
     const uint32_t d_tmem = tmem + kTmemO0 + (x ? 128u : 0u);
+    constexpr int kSteps = kBN / 16 / 2;  // K = 16 keys per instruction
 #pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk) {
+    for (int i = 0; i < kSteps; ++i) {
+        const int kk = half * kSteps + i;
         ptx::mma_ts_elect(d_tmem, p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 2048, L::kBoxBytes, 1024),
-                    kIdesc, (accumulate || kk > 0) ? 1u : 0u);
+                    kIdesc, (accumulate || i > 0) ? 1u : 0u);
     }
 }
 
 // The MMA warp's loop over the pairs of its CTA.  qk(x, slot) issues the score
-// product of tile x from ring slot `slot`; issue(x, slot, accumulate) the P V
-// product.  Shared by the bf16 and the e4m3 kernels.
+// product of tile x from ring slot `slot`; issue(x, slot, half, accumulate) the
+// P V product of key half `half`.  Shared by the bf16 and the e4m3 kernels.
 template <class L, int STAGES, class IssueQK, class IssuePV>
 __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, volatile int* abort_flag,
                                          IssueQK&& qk, IssuePV&& issue) {
@@ -474,25 +482,28 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
     uint32_t f = 0;
     int ring = 0;  // K/V ring slots consumed
     bool ok = true;
-    // Waits for p_ready of tile x; before the first PV of a pair also for the
-    // previous pair's epilogue to have read O.
-    auto pv_ready = [&](int x) -> bool {
-        if (!warp_wait(L::bar_p_ready(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
-        f ^= kPc << x;
+    // P V of tile x in two halves of 64 keys: the first waits for the softmax's
+    // half hand-off (p_half) and, before the first P V of a pair, for the
+    // previous pair's epilogue to have read O (o_free); the second waits for
+    // the whole of P (p_ready).  Both barriers complete once per key block.
+    auto pv = [&](int x, int slot, bool last) -> bool {
+        if (!warp_wait(L::bar_p_half(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
         if ((f & (kFirst << x)) && (f & (kPending << x))) {
             if (!warp_wait(L::bar_o_free(sbase, x), (f >> (4 + x)) & 1u, abort_flag, lim)) return false;
             f ^= (kFreed << x) | (kPending << x);
         }
         ptx::tc_fence_after_sync();
-        return true;
-    };
-    auto pv = [&](int x, int slot, bool last) {
-        issue(x, slot, !(f & (kFirst << x)));
+        issue(x, slot, 0, !(f & (kFirst << x)));
         f &= ~(kFirst << x);
+        if (!warp_wait(L::bar_p_ready(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
+        f ^= kPc << x;
+        ptx::tc_fence_after_sync();
+        issue(x, slot, 1, true);
         if (last) {
             ptx::tc_commit_elect(L::bar_o_done(sbase, x));
             f |= kPending << x;
         }
+        return true;
     };
     while (ok) {
         const int u = unit_take<L>(sbase, (f >> kUnitShift) & 3u, abort_flag, lim);
@@ -518,10 +529,7 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
             }
             if (j > w.ulo) {
                 const int pvs = (ring - 1) % STAGES;
-                if (j - 1 >= lo1 && j - 1 < hi1) {
-                    if (!(ok = pv_ready(1))) break;
-                    pv(1, pvs, j - 1 == hi1 - 1);
-                }
+                if (j - 1 >= lo1 && j - 1 < hi1 && !(ok = pv(1, pvs, j - 1 == hi1 - 1))) break;
                 ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
             }
             if (j >= lo1 && j < hi1) {
@@ -532,19 +540,13 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
             if (j == w.uhi - 1) ptx::tc_commit_elect(L::bar_q_empty(sbase));  // last score products issued
             if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), ((ring + 1) / STAGES) & 1, abort_flag, lim))) break;
             ptx::tc_fence_after_sync();
-            if (j >= lo0 && j < hi0) {
-                if (!(ok = pv_ready(0))) break;
-                pv(0, vs, j == hi0 - 1);
-            }
+            if (j >= lo0 && j < hi0 && !(ok = pv(0, vs, j == hi0 - 1))) break;
         }
         if (!ok) break;
         if (w.uhi > w.ulo) {
             const int j = w.uhi - 1;
             const int vs = (ring - 1) % STAGES;
-            if (j >= lo1 && j < hi1) {
-                if (!(ok = pv_ready(1))) break;
-                pv(1, vs, true);
-            }
+            if (j >= lo1 && j < hi1 && !(ok = pv(1, vs, true))) break;
             ptx::tc_commit_elect(L::bar_kv_empty(sbase, vs));
         } else {
             ptx::tc_commit_elect(L::bar_q_empty(sbase));  // no products: Q is free
@@ -560,7 +562,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
                                          volatile int* abort_flag) {
     mma_loop<SmemLayout<D, STAGES>, STAGES>(
         p, sbase, abort_flag, [&](int x, int slot) { issue_qk<D, STAGES>(tmem, sbase, x, slot); },
-        [&](int x, int slot, bool acc) { issue_pv<D, STAGES>(tmem, sbase, x, slot, acc); });
+        [&](int x, int slot, int half, bool acc) { issue_pv<D, STAGES>(tmem, sbase, x, slot, half, acc); });
 }
 
 // ---------------------------------------------------------------- softmax
@@ -692,6 +694,11 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
                 }
             }
             ptx::tmem_st16(t_p + q * 16, pk);
+            if (q == 1) {  // keys 0..63 of the block: their P V product may start
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before_sync();
+                ptx::mbar_arrive(L::bar_p_half(sbase, x));
+            }
         }
         {
             float a0, a1, b0, b1;
