@@ -99,8 +99,8 @@ struct Layout {
     static constexpr uint32_t kKV = 2 * kTileBytes;
     static constexpr uint32_t kBar = kKV + kStages * kTileBytes;
     // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
-    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_half[2]
-    static constexpr uint32_t kNumBars = 18 + 2 * kStages;
+    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_part[2][kPParts - 1]
+    static constexpr uint32_t kNumBars = 16 + 2 * (kPParts - 1) + 2 * kStages;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem address, abort flag
     static constexpr uint32_t kClcResp = kMisc + 16;        // launch-control response (16 B)
     static constexpr uint32_t kUnitQ = kClcResp + 16;       // unit queue: two ints
@@ -139,8 +139,8 @@ struct Layout {
     static __device__ __forceinline__ uint32_t bar_unit_empty(uint32_t base, int slot) {
         return base + kBar + 8u * (14 + 2 * kStages + slot);
     }
-    static __device__ __forceinline__ uint32_t bar_p_half(uint32_t base, int x) {
-        return base + kBar + 8u * (16 + 2 * kStages + x);
+    static __device__ __forceinline__ uint32_t bar_p_part(uint32_t base, int x, int k) {
+        return base + kBar + 8u * (16 + 2 * kStages + (kPParts - 1) * x + k);
     }
 };
 
@@ -209,16 +209,16 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, i
                         ptx::smem_desc_sw128(ka + kk * 32, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
 }
 
-// Keys [64 half, 64 half + 64) of the block (as in the bf16 kernel).
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot, int half, bool accumulate) {
+// Keys [128 part / kPParts, 128 (part + 1) / kPParts) of the block.
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot, int part, bool accumulate) {
     using L = Layout;
     constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, kD);
     const uint32_t va = sbase + L::kKV + slot * kTileBytes;  // V^T: d rows x 128 keys
     const uint32_t p_tmem = tmem + (x ? 128u : 0u) + kPOffset;
-    constexpr int kSteps = kBN / 32 / 2;  // 32 keys per step = 8 packed columns of P
+    constexpr int kSteps = kBN / 32 / kPParts;  // 32 keys per step = 8 packed columns of P
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
-        const int kk = half * kSteps + i;
+        const int kk = part * kSteps + i;
         mma_ts_f8_elect(tmem + kTmemO0 + (x ? 128u : 0u), p_tmem + kk * 8,
                         ptx::smem_desc_sw128(va + kk * 32, 16, 1024), kIdesc, (accumulate || i > 0) ? 1u : 0u);
     }
@@ -230,7 +230,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
                                          volatile int* abort_flag) {
     mma_loop<Layout, kStages>(
         p, sbase, abort_flag, [&](int x, int slot) { issue_qk(tmem, sbase, x, slot); },
-        [&](int x, int slot, int half, bool acc) { issue_pv(tmem, sbase, x, slot, half, acc); });
+        [&](int x, int slot, int part, bool acc) { issue_pv(tmem, sbase, x, slot, part, acc); });
 }
 
 // One thread per query row, as in the bf16 kernel; P goes to tensor memory as
@@ -340,10 +340,10 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
                     rq1 = add_e4m3x4_to_f32(rq1, pk[i]);
             }
             ptx::tmem_st8(t_p + q * 8, pk);
-            if (q == 1) {  // keys 0..63 of the block: their P V product may start
+            if ((q + 1) % (4 / kPParts) == 0 && q < 3) {  // a part of P is complete
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before_sync();
-                ptx::mbar_arrive(L::bar_p_half(sbase, x));
+                ptx::mbar_arrive(L::bar_p_part(sbase, x, q / (4 / kPParts)));
             }
         }
         {

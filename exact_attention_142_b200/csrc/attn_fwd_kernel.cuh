@@ -70,6 +70,10 @@ constexpr uint32_t kRegsOther = 72;
 // core's at d = 128 and would otherwise be the bottleneck).
 constexpr int kPolyPeriod = 8;
 
+// P is handed to the P V product in kPParts parts of 128 / kPParts keys: the
+// product of one part overlaps the exponentials of the next.
+constexpr int kPParts = 2;
+
 enum : int { kPairHeads = 0, kPairRows = 1 };
 
 // 2^x for a pair of arguments x <= 8 on the FMA/ALU pipes:
@@ -120,8 +124,8 @@ struct SmemLayout {
     static constexpr uint32_t kKV = 2 * kTileBytes;
     static constexpr uint32_t kBar = kKV + STAGES * kTileBytes;
     // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
-    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_half[2]
-    static constexpr uint32_t kNumBars = 18 + 2 * STAGES;
+    // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_part[2][kPParts - 1]
+    static constexpr uint32_t kNumBars = 16 + 2 * (kPParts - 1) + 2 * STAGES;
     static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem address, abort flag
     static constexpr uint32_t kClcResp = kMisc + 16;        // launch-control response (16 B)
     static constexpr uint32_t kUnitQ = kClcResp + 16;       // unit queue: two ints
@@ -162,8 +166,8 @@ struct SmemLayout {
     static __device__ __forceinline__ uint32_t bar_unit_empty(uint32_t base, int slot) {
         return base + kBar + 8u * (14 + 2 * STAGES + slot);
     }
-    static __device__ __forceinline__ uint32_t bar_p_half(uint32_t base, int x) {
-        return base + kBar + 8u * (16 + 2 * STAGES + x);
+    static __device__ __forceinline__ uint32_t bar_p_part(uint32_t base, int x, int k) {
+        return base + kBar + 8u * (16 + 2 * STAGES + (kPParts - 1) * x + k);
     }
 };
 
@@ -366,7 +370,8 @@ __device__ __forceinline__ void init_schedule_barriers(uint32_t sbase) {
     ptx::mbar_init(L::bar_q_empty(sbase), 1);
     for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_o_free(sbase, x), 128);
     ptx::mbar_init(L::bar_clc(sbase), 1);
-    for (int x = 0; x < 2; ++x) ptx::mbar_init(L::bar_p_half(sbase, x), 128);
+    for (int x = 0; x < 2; ++x)
+        for (int k = 0; k < kPParts - 1; ++k) ptx::mbar_init(L::bar_p_part(sbase, x, k), 128);
     for (int slot = 0; slot < 2; ++slot) {
         ptx::mbar_init(L::bar_unit_full(sbase, slot), 1);
         ptx::mbar_init(L::bar_unit_empty(sbase, slot), kUnitReaders);
@@ -441,10 +446,9 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, i
     }
 }
 
-// Keys [64 half, 64 half + 64) of the block: the softmax hands P over in two
-// halves, so the first half's product overlaps the second half's exponentials.
+// Keys [128 part / kPParts, 128 (part + 1) / kPParts) of the block.
 template <int D, int STAGES>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot, int half,
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, int slot, int part,
                                          bool accumulate) {
     using L = SmemLayout<D, STAGES>;
     // B = V is [keys, d] with d contiguous: MN-major operand.  Swizzle atoms of
@@ -454,18 +458,18 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
     const uint32_t va = sbase + L::kKV + slot * L::kTileBytes;
     const uint32_t p_tmem = tmem + (x ? 128u : 0u) + kPOffset;
     const uint32_t d_tmem = tmem + kTmemO0 + (x ? 128u : 0u);
-    constexpr int kSteps = kBN / 16 / 2;  // K = 16 keys per instruction
+    constexpr int kSteps = kBN / 16 / kPParts;  // K = 16 keys per instruction
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
-        const int kk = half * kSteps + i;
+        const int kk = part * kSteps + i;
         ptx::mma_ts_elect(d_tmem, p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 2048, L::kBoxBytes, 1024),
                     kIdesc, (accumulate || i > 0) ? 1u : 0u);
     }
 }
 
 // The MMA warp's loop over the pairs of its CTA.  qk(x, slot) issues the score
-// product of tile x from ring slot `slot`; issue(x, slot, half, accumulate) the
-// P V product of key half `half`.  Shared by the bf16 and the e4m3 kernels.
+// product of tile x from ring slot `slot`; issue(x, slot, part, accumulate) the
+// P V product of key part `part`.  Shared by the bf16 and the e4m3 kernels.
 template <class L, int STAGES, class IssueQK, class IssuePV>
 __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, volatile int* abort_flag,
                                          IssueQK&& qk, IssuePV&& issue) {
@@ -482,23 +486,24 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
     uint32_t f = 0;
     int ring = 0;  // K/V ring slots consumed
     bool ok = true;
-    // P V of tile x in two halves of 64 keys: the first waits for the softmax's
-    // half hand-off (p_half) and, before the first P V of a pair, for the
-    // previous pair's epilogue to have read O (o_free); the second waits for
-    // the whole of P (p_ready).  Both barriers complete once per key block.
+    // P V of tile x in kPParts parts: part k waits for the softmax's hand-off of
+    // that part (p_part, the last one p_ready); before the first P V of a pair
+    // the first part also waits for the previous pair's epilogue to have read O
+    // (o_free).  Every hand-off barrier completes once per key block.
     auto pv = [&](int x, int slot, bool last) -> bool {
-        if (!warp_wait(L::bar_p_half(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
-        if ((f & (kFirst << x)) && (f & (kPending << x))) {
-            if (!warp_wait(L::bar_o_free(sbase, x), (f >> (4 + x)) & 1u, abort_flag, lim)) return false;
-            f ^= (kFreed << x) | (kPending << x);
+#pragma unroll
+        for (int k = 0; k < kPParts; ++k) {
+            const uint32_t bar = k < kPParts - 1 ? L::bar_p_part(sbase, x, k) : L::bar_p_ready(sbase, x);
+            if (!warp_wait(bar, (f >> x) & 1u, abort_flag, lim)) return false;
+            if (k == 0 && (f & (kFirst << x)) && (f & (kPending << x))) {
+                if (!warp_wait(L::bar_o_free(sbase, x), (f >> (4 + x)) & 1u, abort_flag, lim)) return false;
+                f ^= (kFreed << x) | (kPending << x);
+            }
+            ptx::tc_fence_after_sync();
+            issue(x, slot, k, k > 0 || !(f & (kFirst << x)));
         }
-        ptx::tc_fence_after_sync();
-        issue(x, slot, 0, !(f & (kFirst << x)));
         f &= ~(kFirst << x);
-        if (!warp_wait(L::bar_p_ready(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
         f ^= kPc << x;
-        ptx::tc_fence_after_sync();
-        issue(x, slot, 1, true);
         if (last) {
             ptx::tc_commit_elect(L::bar_o_done(sbase, x));
             f |= kPending << x;
@@ -562,7 +567,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
                                          volatile int* abort_flag) {
     mma_loop<SmemLayout<D, STAGES>, STAGES>(
         p, sbase, abort_flag, [&](int x, int slot) { issue_qk<D, STAGES>(tmem, sbase, x, slot); },
-        [&](int x, int slot, int half, bool acc) { issue_pv<D, STAGES>(tmem, sbase, x, slot, half, acc); });
+        [&](int x, int slot, int part, bool acc) { issue_pv<D, STAGES>(tmem, sbase, x, slot, part, acc); });
 }
 
 // ---------------------------------------------------------------- softmax
@@ -694,10 +699,10 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
                 }
             }
             ptx::tmem_st16(t_p + q * 16, pk);
-            if (q == 1) {  // keys 0..63 of the block: their P V product may start
+            if ((q + 1) % (4 / kPParts) == 0 && q < 3) {  // a part of P is complete
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before_sync();
-                ptx::mbar_arrive(L::bar_p_half(sbase, x));
+                ptx::mbar_arrive(L::bar_p_part(sbase, x, q / (4 / kPParts)));
             }
         }
         {
