@@ -590,8 +590,11 @@ def run_torch_sdpa(args, w: W.Workload):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     fl = flops_of(w)
     results = {}
-    for name, be in [("flash", SDPBackend.FLASH_ATTENTION), ("cudnn", SDPBackend.CUDNN_ATTENTION),
-                     ("efficient", SDPBackend.EFFICIENT_ATTENTION)]:
+    backends = [("flash", SDPBackend.FLASH_ATTENTION), ("cudnn", SDPBackend.CUDNN_ATTENTION),
+                ("efficient", SDPBackend.EFFICIENT_ATTENTION)]
+    for name, be in backends:
+        if args.sdpa_backend not in ("all", name):
+            continue
         try:
             with sdpa_kernel([be]):
                 def call():
@@ -1191,6 +1194,8 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference", "torch_sdpa"],
                     help="torch_sdpa: context only, PyTorch's scaled_dot_product_attention on the "
                          "same dense workload (not this library; one GPU)")
+    ap.add_argument("--sdpa-backend", default="all", choices=["all", "cudnn", "flash", "efficient"],
+                    help="--impl torch_sdpa only: the backends to time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
