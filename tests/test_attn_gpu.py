@@ -309,3 +309,22 @@ def test_schedule_accumulate_many_pairs():
     # fp32 output: only the weights' bf16 rounding remains (no output rounding)
     assert float(np.abs(o_acc.cpu().double().numpy() - o_ref.reshape(B, N, Hq, d)).max()) <= 5e-3
     assert float(np.abs(l_acc.cpu().double().numpy() - lse_ref.reshape(B, Hq, N)).max()) <= TOL_LSE
+
+
+def test_long_sequence_sampled_rows():
+    """A 131 072-token causal sequence (GQA 8:1): offsets past 2^31 bytes in O and
+    the deepest key ranges, checked on sampled rows."""
+    B, Hq, Hkv, N, d = 1, 8, 1, 131072, 128
+    q, k, v = W.draw_qkv((B, N, Hq, d), (B, N, Hkv, d), 51)
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=True)
+    o, lse = gpu_run(q, k, v, **kw)
+    rows = sample_rows([N], Hq, n_random=120, seed=52)
+    rows = np.concatenate([rows, np.array([[0, Hq - 1, N - 1], [0, 0, N - 129], [0, 3, N // 2 + 127]])])
+    o_ref, lse_ref, _ = oracle_run(q, k, v, rows=rows, **kw)
+    of = o.reshape(-1, Hq, d)
+    lf = lse.reshape(-1)
+    got_o = np.stack([of[i, h].to(torch.float64).numpy() for b, h, i in rows])
+    got_l = np.array([float(lf[(b * Hq + h) * N + i]) for b, h, i in rows])
+    assert np.abs(got_o - o_ref).max() <= TOL_O
+    assert np.abs(got_l - lse_ref).max() <= TOL_LSE
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()

@@ -126,3 +126,23 @@ def test_bwd_causal_mha_workload_one_head():
     ref = ref_bwd(sub(q), sub(k), sub(v), sub(do), B=1, Hq=1, Hkv=1, N=w.N, d=w.d,
                   scale=w.scale, causal=True)
     compare((dq[b:b + 1, :, h:h + 1], dk[b:b + 1, :, h:h + 1], dv[b:b + 1, :, h:h + 1]), ref)
+
+
+def test_bwd_causal_gqa_workload_one_group():
+    """The benchmark's causal GQA workload (B=2, Hq=32, Hkv=8, N=8192, d=128) on
+    the GPU; the oracle checks sequence 1, K/V head 5 with its four query heads
+    (a sub-problem whose gradients depend only on its own q, k, v, dout)."""
+    w = W.workload(3)
+    q, k, v = W.inputs(w)
+    g = torch.Generator().manual_seed(w.seed + 1000)
+    do = torch.randn(q.shape, dtype=torch.float32, generator=g).to(torch.bfloat16)
+    kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d, scale=w.scale, causal=True)
+    dq, dk, dv = gpu_bwd(q, k, v, do, **kw)
+    b, gkv = 1, 5
+    grp = w.Hq // w.Hkv
+    hs = slice(gkv * grp, (gkv + 1) * grp)
+    subq = lambda t: t[b:b + 1, :, hs].contiguous()
+    subk = lambda t: t[b:b + 1, :, gkv:gkv + 1].contiguous()
+    ref = ref_bwd(subq(q), subk(k), subk(v), subq(do), B=1, Hq=grp, Hkv=1, N=w.N, d=w.d,
+                  scale=w.scale, causal=True)
+    compare((dq[b:b + 1, :, hs], dk[b:b + 1, :, gkv:gkv + 1], dv[b:b + 1, :, gkv:gkv + 1]), ref)
