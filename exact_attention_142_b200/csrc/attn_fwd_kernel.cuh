@@ -735,6 +735,7 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
         // both log-sum-exps in log2 units; weights relative to the larger one
         const float lse_new = l_sum > 0.0f ? m_ref + ptx::lg2_approx(l_sum) : -INFINITY;
         const float lse_old = store ? p.lse[idx] * kLog2e : -INFINITY;
+        const bool has_old = lse_old != -INFINITY;  // an empty row's o_acc is not read
         const float mx = fmaxf(lse_old, lse_new);
         const float mu = mx == -INFINITY ? 0.0f : mx;
         const float w_old = ptx::ex2_approx(lse_old - mu);
@@ -752,7 +753,7 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
                     float4* ap = reinterpret_cast<float4*>(acc + cc * 32 + v * 4);
-                    float4 a = *ap;
+                    float4 a = has_old ? *ap : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                     a.x = fmaf(a_old, a.x, a_new * __uint_as_float(o[4 * v + 0]));
                     a.y = fmaf(a_old, a.y, a_new * __uint_as_float(o[4 * v + 1]));
                     a.z = fmaf(a_old, a.z, a_new * __uint_as_float(o[4 * v + 2]));

@@ -92,7 +92,8 @@ def ring_attention_forward(q_chunks: Sequence, k_chunks: Sequence, v_chunks: Seq
         accumulate = cuda_accumulate(scale, stream)
     q_chunks = list(q_chunks)
     B, C, Hq, d = q_chunks[0].shape
-    o_acc = [torch.zeros((B, C, Hq, d), dtype=torch.float32, device=q.device) for q in q_chunks]
+    # rows whose LSE is -inf are empty: their O is neither read nor needs zeroing
+    o_acc = [torch.empty((B, C, Hq, d), dtype=torch.float32, device=q.device) for q in q_chunks]
     lse_acc = [torch.full((B, Hq, C), float("-inf"), dtype=torch.float32, device=q.device)
                for q in q_chunks]
     cur_k, cur_v = list(k_chunks), list(v_chunks)

@@ -120,7 +120,8 @@ size_t attn_fwd_fp8_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int pa
  * "How it works", Step 3).
  *   o_acc   [tokens, Hq, d] fp32 and lse_acc (laid out like lse) hold a
  *           partial result over some other keys; a row whose lse_acc is -inf
- *           holds nothing yet (start from o_acc = 0, lse_acc = -inf).
+ *           holds nothing yet, and its o_acc values are not read (start from
+ *           lse_acc = -inf; o_acc may then be uninitialised).
  * With (O', L') this call's attention of q over k, v (natural-log LSE), each
  * row becomes  L = log(e^lse_acc + e^L'),
  *              o_acc = (e^lse_acc o_acc + e^L' O') / e^L,   lse_acc = L,

@@ -63,7 +63,9 @@ def _oracle_step(B, Hq, Hkv, d, scale):
         # weights [B, Hq, C] -> [B, C, Hq, 1]
         wo = np.transpose(w_old, (0, 2, 1))[..., None]
         wn = np.transpose(w_new, (0, 2, 1))[..., None]
-        acc = o_acc.to(torch.float64).numpy()
+        # a row whose accumulator LSE is -inf is empty: its O is not read
+        empty = np.transpose(np.isneginf(old_l), (0, 2, 1))[..., None]
+        acc = np.where(empty, 0.0, o_acc.to(torch.float64).numpy())
         o_acc.copy_(torch.from_numpy(wo * acc + wn * o))
         lse_acc.copy_(torch.from_numpy(L))
     return step

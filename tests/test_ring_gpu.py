@@ -118,3 +118,22 @@ def test_acc_to_bf16_rounds_to_nearest_even():
     ea.attn_acc_to_bf16(xd, out, n)
     torch.cuda.synchronize()
     assert torch.equal(out[:n].cpu().view(torch.int16), x.to(torch.bfloat16).view(torch.int16))
+
+
+def test_accumulate_ignores_empty_rows_contents():
+    """A row whose accumulator LSE is -inf is empty: whatever its O holds (NaN
+    here) is not read, so an unzeroed accumulator gives the attention output."""
+    B, N, Hq, Hkv, d = 1, 300, 4, 2, 128
+    q, k, v = W.draw_qkv((B, N, Hq, d), (B, N, Hkv, d), seed=9)
+    scale = default_scale(d)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o_acc = torch.full((B, N, Hq, d), float("nan"), dtype=torch.float32, device=DEV)
+    l_acc = torch.full((B, Hq, N), float("-inf"), dtype=torch.float32, device=DEV)
+    ea.attn_fwd_accumulate(qd, kd, vd, o_acc, l_acc, B, Hq, Hkv, N, d, scale, True)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    o_ref, lse_ref = ref(q, k, v, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=scale, causal=True)
+    got = o_acc.cpu().double().numpy()
+    assert np.isfinite(got).all()
+    assert float(np.abs(got - o_ref).max()) <= 5e-3
+    assert float(np.abs(l_acc.cpu().double().numpy() - lse_ref).max()) <= TOL_LSE
