@@ -1,11 +1,14 @@
 // attn_fwd_kernel.cuh -- fused exact attention forward for sm_100a.
 //
-// One CTA owns two 128-row query tiles that read the same key/value head and
-// streams 128-key blocks of K and V through a shared-memory ring:
+// A CTA computes pairs of 128-row query tiles that read the same key/value
+// head, streaming 128-key blocks of K and V through a shared-memory ring.  It
+// is persistent: after its own pair it takes over the pairs of CTAs that have
+// not started (cluster launch control; see UnitSource).
 //
 //   warps 0-3  softmax for query tile 0 (one thread per query row)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    producer: TMA loads of Q (once) and of the K/V ring
+//   warp  8    producer: the schedule, TMA loads of Q (once per pair) and of
+//              the K/V ring
 //   warp  9    MMA issuer: tcgen05 S = Q K^T (both operands in shared memory)
 //              and O += P V (P read from tensor memory)
 //   (both run converged over all 32 lanes; one elected lane issues)
