@@ -128,6 +128,13 @@ __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]
         : "memory");
 }
 
+// One arrival per elementwise warp, after every lane's tensor-memory stores
+// are complete and fenced.
+__device__ __forceinline__ void elem_warp_arrive(uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
+}
+
 struct Seq {
     int start, len;
 };
@@ -464,7 +471,7 @@ __device__ __forceinline__ void dkv_elementwise(const DkvWork& w, const BwdParam
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(L::bar_p(sbase, t & 1));
+        elem_warp_arrive(L::bar_p(sbase, t & 1));
     }
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
@@ -519,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(L::bar_st(sbase, b), 1);
-            ptx::mbar_init(L::bar_p(sbase, b), kElemThreads);
+            ptx::mbar_init(L::bar_p(sbase, b), kElemWarps);
         }
         ptx::mbar_init(L::bar_done(sbase), 1);
         *abort_flag = 0;
@@ -754,7 +761,7 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
         dq_stage_a<D, STAGES>(tl, sbase, x, row);
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(L::bar_a(sbase));
+        elem_warp_arrive(L::bar_a(sbase));
     }
     for (int n = w.n_lo; ok && n < w.n_hi; ++n) {
         const int t = n - w.n_lo;
@@ -784,7 +791,7 @@ __device__ __forceinline__ void dq_elementwise(const DqWork& w, const BwdParams&
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before_sync();
-        ptx::mbar_arrive(L::bar_ds(sbase, t & 1));
+        elem_warp_arrive(L::bar_ds(sbase, t & 1));
     }
     if (!ok) return;
     if (!__all_sync(0xffffffffu, bounded_wait(L::bar_done(sbase), 0, abort_flag, lim))) return;
@@ -831,10 +838,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(L::bar_st(sbase, b), 1);
-            ptx::mbar_init(L::bar_ds(sbase, b), kElemThreads);
+            ptx::mbar_init(L::bar_ds(sbase, b), kElemWarps);
         }
         ptx::mbar_init(L::bar_done(sbase), 1);
-        ptx::mbar_init(L::bar_a(sbase), kElemThreads);
+        ptx::mbar_init(L::bar_a(sbase), kElemWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_q);
