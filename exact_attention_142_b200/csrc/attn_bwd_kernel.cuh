@@ -57,7 +57,6 @@ constexpr int kGroupCols = kStep / kGroups;  // columns of a step per group (16)
 constexpr int kWarpProducer = kElemWarps;
 constexpr int kWarpMma = kElemWarps + 1;
 constexpr int kThreads = (kElemWarps + 2) * 32;
-constexpr int kElemThreads = kElemWarps * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBox128 = 128 * 128;  // TMA box of a 128-row tile: 128 rows x 128 bytes
 constexpr uint32_t kBox64 = 64 * 128;    // TMA box of a 64-row step tile
