@@ -22,7 +22,9 @@ def attention(q, k, v, *, causal=False, window_left=-1, window_right=-1, scale=N
 
     Dense: q [B, N, Hq, d], k/v [B, N, Hkv, d] -> o [B, N, Hq, d], lse [B, Hq, N].
     Packed: q [T, Hq, d], k/v [T, Hkv, d], cu_seqlens int32 [B+1] on the device
-    -> o [T, Hq, d], lse [Hq, T].
+    -> o [T, Hq, d], lse [Hq, T].  Without max_seqlen the longest sequence is
+    read back from cu_seqlens (a device-to-host copy); attn_fwd itself never
+    reads cu_seqlens on the host.
     """
     import math
 
@@ -36,6 +38,8 @@ def attention(q, k, v, *, causal=False, window_left=-1, window_right=-1, scale=N
         Hkv = k.shape[1]
         B = cu_seqlens.numel() - 1
         lse = torch.empty((Hq, N), dtype=torch.float32, device=q.device)
+        if max_seqlen <= 0 and B > 0:
+            max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item())
     o = torch.empty_like(q)
     if scale is None:
         scale = 1.0 / math.sqrt(d)

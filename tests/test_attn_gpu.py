@@ -328,3 +328,24 @@ def test_long_sequence_sampled_rows():
     assert np.abs(got_o - o_ref).max() <= TOL_O
     assert np.abs(got_l - lse_ref).max() <= TOL_LSE
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def test_attention_convenience_dense_and_packed():
+    """ea.attention allocates the outputs; packed batches without max_seqlen."""
+    d, Hq, Hkv = 128, 4, 2
+    q, k, v = W.draw_qkv((2, 200, Hq, d), (2, 200, Hkv, d), 61)
+    o, lse = ea.attention(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    torch.cuda.synchronize()
+    o_ref, lse_ref, _ = oracle_run(q, k, v, B=2, Hq=Hq, Hkv=Hkv, N=200, d=d, scale=default_scale(d),
+                                   causal=True)
+    compare_full(o.cpu(), lse.cpu(), o_ref, lse_ref)
+    lengths = [5, 0, 300, 130]
+    cu = W.cumulative(lengths)
+    T = cu[-1]
+    q, k, v = W.draw_qkv((T, Hq, d), (T, Hkv, d), 62)
+    o, lse = ea.attention(q.cuda(), k.cuda(), v.cuda(), causal=True,
+                          cu_seqlens=torch.tensor(cu, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    o_ref, lse_ref, _ = oracle_run(q, k, v, B=len(lengths), Hq=Hq, Hkv=Hkv, N=T, d=d,
+                                   scale=default_scale(d), causal=True, cu_seqlens=cu)
+    compare_full(o.cpu(), lse.cpu(), o_ref, lse_ref)
