@@ -439,14 +439,18 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, i
     const uint32_t qa = sbase + (x ? L::kQ1 : L::kQ0);
     const uint32_t ka = sbase + L::kKV + slot * L::kTileBytes;
     const uint32_t d_tmem = tmem + (x ? 128u : 0u);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        // K-major, 128-byte swizzle: 16 elements (32 bytes) per step inside a
-        // 64-element box, the next box 16 KB further.
-        const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
-        ptx::mma_ss_elect(d_tmem, ptx::smem_desc_sw128(qa + off, 16, 1024),
-                    ptx::smem_desc_sw128(ka + off, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
-    }
+    // K-major, 128-byte swizzle: 16 elements (32 bytes) per step inside a
+    // 64-element box, the next box 16 KB further.  A step's descriptor is the
+    // tile's plus the byte offset / 16 (the 14-bit start-address field cannot
+    // carry: shared addresses stay below 256 KB).  All steps go out from one
+    // elected lane.
+    static_assert(L::kBoxBytes == 16384, "the step offsets assume 16 KB boxes");
+    const uint64_t qd = ptx::smem_desc_sw128(qa, 16, 1024);
+    const uint64_t kd = ptx::smem_desc_sw128(ka, 16, 1024);
+    if constexpr (D == 128)
+        ptx::mma_ss_kmajor8_elect(d_tmem, qd, kd, kIdesc, 0u);
+    else
+        ptx::mma_ss_kmajor4_elect(d_tmem, qd, kd, kIdesc, 0u);
 }
 
 // Keys [128 part / kPParts, 128 (part + 1) / kPParts) of the block.
@@ -462,12 +466,12 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
     const uint32_t p_tmem = tmem + (x ? 128u : 0u) + kPOffset;
     const uint32_t d_tmem = tmem + kTmemO0 + (x ? 128u : 0u);
     constexpr int kSteps = kBN / 16 / kPParts;  // K = 16 keys per instruction
-#pragma unroll
-    for (int i = 0; i < kSteps; ++i) {
-        const int kk = part * kSteps + i;
-        ptx::mma_ts_elect(d_tmem, p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 2048, L::kBoxBytes, 1024),
-                    kIdesc, (accumulate || i > 0) ? 1u : 0u);
-    }
+    static_assert(kSteps == 4, "one four-step group per part");
+    // Step kk reads P columns +8 kk and the V rows 16 kk.. (2 KB further each).
+    const int kk0 = part * kSteps;
+    ptx::mma_ts_mnmajor4_elect(d_tmem, p_tmem + kk0 * 8,
+                               ptx::smem_desc_sw128(va, L::kBoxBytes, 1024) + ((kk0 * 2048) >> 4), kIdesc,
+                               accumulate ? 1u : 0u);
 }
 
 // The MMA warp's loop over the pairs of its CTA.  qk(x, slot) issues the score
