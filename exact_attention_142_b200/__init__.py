@@ -7,13 +7,15 @@ outputs with torch and calls ``attn_fwd``.
 """
 from ._binding import (  # noqa: F401
     ATTN_ERR_ALIGN, ATTN_ERR_CUDA, ATTN_ERR_DEVICE_TIMEOUT, ATTN_ERR_NULL, ATTN_ERR_PAGE, ATTN_ERR_SCALE,
-    ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WINDOW, ATTN_ERR_WORKSPACE, ATTN_OK, AttnError,
-    ATTN_DECODE_NOALLOC_SCRATCH_BYTES, attn_bwd, attn_bwd_workspace_bytes, attn_decode,
+    ATTN_ERR_SEQLENS, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WINDOW, ATTN_ERR_WORKSPACE,
+    ATTN_OK, AttnError, attn_bwd, attn_bwd_workspace_bytes, attn_decode,
     attn_decode_default_splits,
-    attn_decode_noalloc, attn_decode_workspace_bytes, attn_device_status,
+    attn_decode_noalloc, attn_decode_noalloc_scratch_bytes, attn_decode_workspace_bytes,
+    attn_device_status,
     attn_acc_to_bf16, attn_fwd, attn_fwd_accumulate, attn_fwd_fp8, attn_fwd_fp8_workspace_bytes,
     attn_fwd_host, attn_fwd_host_workspace_bytes,
-    attn_selftest_bounded_wait, attn_status_string, library_path, load_library)
+    attn_selftest_bounded_wait, attn_selftest_exp2_poly, attn_status_string, library_path,
+    load_library)
 
 
 def attention(q, k, v, *, causal=False, window_left=-1, window_right=-1, scale=None,

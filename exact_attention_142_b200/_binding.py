@@ -26,6 +26,7 @@ ATTN_ERR_SCALE = -7
 ATTN_ERR_WORKSPACE = -8
 ATTN_ERR_DEVICE_TIMEOUT = -9
 ATTN_ERR_PAGE = -10
+ATTN_ERR_SEQLENS = -11
 
 
 class AttnError(RuntimeError):
@@ -76,6 +77,8 @@ def load_library():
         lib.attn_decode_noalloc.restype = I
         lib.attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,
                                             I, I, P]
+        lib.attn_decode_noalloc_scratch_bytes.restype = S
+        lib.attn_decode_noalloc_scratch_bytes.argtypes = []
         lib.attn_decode_workspace_bytes.restype = S
         lib.attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
         lib.attn_decode_default_splits.restype = I
@@ -86,6 +89,8 @@ def load_library():
         lib.attn_device_status.argtypes = []
         lib.attn_selftest_bounded_wait.restype = I
         lib.attn_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
+        lib.attn_selftest_exp2_poly.restype = I
+        lib.attn_selftest_exp2_poly.argtypes = [P, P, ctypes.c_longlong, P]
         _lib = lib
         return lib
 
@@ -218,7 +223,6 @@ def attn_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, 
     return rc
 
 
-ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv, Nq,
@@ -238,6 +242,11 @@ def attn_decode_noalloc(q, k_cache, v_cache, o, lse, cache_seqlens, block_table,
     if check and rc != ATTN_OK:
         raise AttnError(rc, "attn_decode_noalloc")
     return rc
+
+
+def attn_decode_noalloc_scratch_bytes() -> int:
+    """Size of the library's fixed decode scratch array, read from the library."""
+    return int(load_library().attn_decode_noalloc_scratch_bytes())
 
 
 def attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, page_size, pages_per_seq, num_splits) -> int:
@@ -261,3 +270,11 @@ def attn_device_status() -> int:
 
 def attn_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
     return int(load_library().attn_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+def attn_selftest_exp2_poly(x, y, n, stream=None, check=True) -> int:
+    """y = 2^x through the kernels' FMA-pipe exponential (see include/attn.h)."""
+    rc = int(load_library().attn_selftest_exp2_poly(_ptr(x), _ptr(y), int(n), _stream(stream)))
+    if check and rc != ATTN_OK:
+        raise AttnError(rc, "attn_selftest_exp2_poly")
+    return rc

@@ -410,6 +410,8 @@ extern "C" const char* attn_status_string(int status) {
         case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out; outputs are undefined";
         case ATTN_ERR_PAGE: return "a page-table entry lies outside the cache; outputs are undefined";
+        case ATTN_ERR_SEQLENS:
+            return "cu_seqlens do not fit N or max_seqlen; the sequences concerned were skipped";
         default: return "unknown status";
     }
 }
@@ -430,5 +432,34 @@ extern "C" int attn_selftest_bounded_wait(uint64_t limit_ns, struct CUstream_st*
     if (limit_ns > 2000000000ull) limit_ns = 2000000000ull;
     attn::selftest_bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         (unsigned long long)limit_ns);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+namespace {
+
+// y = 2^x through the forward kernels' FMA-pipe exponential, two values per
+// thread (the kernels evaluate it on pairs).
+__global__ void selftest_exp2_poly_kernel(const float* x, float* y, long long n) {
+    const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 2;
+    if (i >= n) return;
+    const bool two = i + 1 < n;
+    float y0, y1;
+    attn::exp2_poly_pair(x[i], two ? x[i + 1] : 0.0f, y0, y1);
+    y[i] = y0;
+    if (two) y[i + 1] = y1;
+}
+
+}  // namespace
+
+extern "C" int attn_selftest_exp2_poly(const float* x, float* y, long long n, struct CUstream_st* stream) {
+    if (n < 0) return ATTN_ERR_SHAPE;
+    if (n == 0) return ATTN_OK;
+    if (!x || !y) return ATTN_ERR_NULL;
+    if (!aligned(x, 4) || !aligned(y, 4)) return ATTN_ERR_ALIGN;
+    const long long blocks = ((n + 1) / 2 + 255) / 256;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+    const int rc = prepare_device(0);
+    if (rc != ATTN_OK) return rc;
+    selftest_exp2_poly_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

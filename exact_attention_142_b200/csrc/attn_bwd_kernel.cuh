@@ -138,11 +138,18 @@ struct Seq {
     int start, len;
 };
 
+// Packed boundaries outside [0, N], decreasing, or longer than the blocks the
+// launch was sized for (max_seqlen) give an empty sequence: nothing of it is
+// read or written, and the block's first thread reports it.
 __device__ __forceinline__ Seq seq_of(const BwdParams& p, int b) {
     Seq s;
     if (p.cu_seqlens) {
-        s.start = p.cu_seqlens[b];
-        s.len = p.cu_seqlens[b + 1] - s.start;
+        const int s0 = p.cu_seqlens[b];
+        const int s1 = p.cu_seqlens[b + 1];
+        const bool bad = s0 < 0 || s1 < s0 || s1 > p.N || (long long)(s1 - s0) > (long long)p.n_blocks * kBN;
+        if (bad && threadIdx.x == 0) atomicCAS(&g_bwd_status, 0, ATTN_ERR_SEQLENS);
+        s.start = bad ? 0 : s0;
+        s.len = bad ? 0 : s1 - s0;
     } else {
         s.start = b * p.N;
         s.len = p.N;

@@ -223,12 +223,15 @@ extern "C" size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, in
     return decode_workspace(B, Hq, Nq, d, plan.splits);
 }
 
-extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
-                           float* lse, const int32_t* cache_seqlens, const int32_t* block_table,
-                           int B, int Hq, int Hkv, int Nq, int d, int page_size, int pages_per_seq,
-                           int num_pages, float scale, int causal, int window_left,
-                           int window_right, int num_splits, void* workspace,
-                           size_t workspace_bytes, struct CUstream_st* stream) {
+namespace {
+
+// Every host-side check of attn_decode's arguments except the workspace; on
+// success `plan` holds the launch plan and `need` the workspace it needs.
+int validate_decode(const void* q, const void* k_cache, const void* v_cache, const void* o,
+                    const float* lse, const int32_t* cache_seqlens, const int32_t* block_table,
+                    int B, int Hq, int Hkv, int Nq, int d, int page_size, int pages_per_seq,
+                    int num_pages, float scale, int window_left, int window_right, int num_splits,
+                    DecodePlan* plan, size_t* need) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || page_size <= 0 || pages_per_seq <= 0 ||
         num_pages <= 0 || num_splits <= 0 || B > 65535)
         return ATTN_ERR_SHAPE;
@@ -242,11 +245,27 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
         return ATTN_ERR_ALIGN;
-    DecodePlan plan;
-    int rc = plan_decode(Hq, Hkv, Nq, page_size, pages_per_seq, num_splits, &plan);
+    const int rc = plan_decode(Hq, Hkv, Nq, page_size, pages_per_seq, num_splits, plan);
     if (rc != ATTN_OK) return rc;
-    if ((long long)Hkv * plan.head_chunks > 65535) return ATTN_ERR_SHAPE;
-    const size_t need = decode_workspace(B, Hq, Nq, d, plan.splits);
+    if ((long long)Hkv * plan->head_chunks > 65535) return ATTN_ERR_SHAPE;
+    *need = decode_workspace(B, Hq, Nq, d, plan->splits);
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                           float* lse, const int32_t* cache_seqlens, const int32_t* block_table,
+                           int B, int Hq, int Hkv, int Nq, int d, int page_size, int pages_per_seq,
+                           int num_pages, float scale, int causal, int window_left,
+                           int window_right, int num_splits, void* workspace,
+                           size_t workspace_bytes, struct CUstream_st* stream) {
+    DecodePlan plan;
+    size_t need = 0;
+    int rc = validate_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv,
+                             Nq, d, page_size, pages_per_seq, num_pages, scale, window_left,
+                             window_right, num_splits, &plan, &need);
+    if (rc != ATTN_OK) return rc;
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
         return ATTN_ERR_WORKSPACE;
     rc = prepare_device();
@@ -315,7 +334,10 @@ int noalloc_scratch(void** out) {
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_ptr[dev]) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();  // leave no pending error for the caller's next CUDA call
+            return ATTN_ERR_CUDA;
+        }
         g_noalloc_ptr[dev] = p;
     }
     *out = g_noalloc_ptr[dev];
@@ -330,14 +352,21 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
                                    int d, int page_size, int pages_per_seq, int num_pages,
                                    float scale, int causal, int window_left, int window_right,
                                    int num_splits, struct CUstream_st* stream) {
-    // Host arithmetic only: 0 for a single slice (no scratch) or invalid sizes,
-    // which attn_decode then rejects with its own status.
-    const size_t need = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, page_size, pages_per_seq,
-                                                    num_splits);
+    // Every argument is checked, and the device is found supported, before
+    // the array's address is looked up: a bad call or an unsupported device
+    // returns attn_decode's own status and touches nothing.
+    DecodePlan plan;
+    size_t need = 0;
+    int rc = validate_decode(q, k_cache, v_cache, o, lse, cache_seqlens, block_table, B, Hq, Hkv,
+                             Nq, d, page_size, pages_per_seq, num_pages, scale, window_left,
+                             window_right, num_splits, &plan, &need);
+    if (rc != ATTN_OK) return rc;
     if (need > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+    rc = prepare_device();
+    if (rc != ATTN_OK) return rc;
     void* scratch = nullptr;
     if (need > 0) {
-        const int rc = noalloc_scratch(&scratch);
+        rc = noalloc_scratch(&scratch);
         if (rc != ATTN_OK) return rc;
     }
     // Every scratch entry the merge kernel reads is written by the slice kernel
@@ -346,4 +375,8 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
                        page_size, pages_per_seq, num_pages, scale, causal, window_left,
                        window_right, num_splits, scratch,
                        need > 0 ? (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
+extern "C" size_t attn_decode_noalloc_scratch_bytes(void) {
+    return (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES;
 }

@@ -145,10 +145,13 @@ struct Layout {
 };
 
 // First padded column of sequence b in V^T (each sequence rounded up to 128).
-__device__ __forceinline__ int vt_start(const FwdParams& p, int b) {
-    if (!p.cu_seqlens) return b * ((p.N + kBN - 1) / kBN) * kBN;
-    int s = 0;
-    for (int i = 0; i < b; ++i) s += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + kBN - 1) / kBN * kBN;
+__device__ __forceinline__ long long vt_start(const FwdParams& p, int b) {
+    if (!p.cu_seqlens) return (long long)b * ((p.N + kBN - 1) / kBN) * kBN;
+    long long s = 0;
+    for (int i = 0; i < b; ++i) {
+        const long long len = (long long)p.cu_seqlens[i + 1] - p.cu_seqlens[i];
+        if (len > 0) s += (len + kBN - 1) / kBN * kBN;
+    }
     return s;
 }
 
@@ -476,11 +479,18 @@ __global__ void __launch_bounds__(256) attn_vt_transpose_kernel(const uint8_t* v
     __shared__ uint8_t tile[64][kD + 4];
     const int b = blockIdx.z, g = blockIdx.y;
     const int start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.N;
-    const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - start : p.N;
+    const int end = p.cu_seqlens ? p.cu_seqlens[b + 1] : start + p.N;
+    // boundaries that do not fit the call: nothing is read or written here (the
+    // attention kernel skips the sequence and reports it)
+    if (start < 0 || end < start || end > (p.cu_seqlens ? p.N : p.B * p.N) ||
+        (long long)(end - start) > (long long)p.n_row_blocks * kBM)
+        return;
+    const int len = end - start;
     const int padded = (len + kBN - 1) / kBN * kBN;
     const int k0 = blockIdx.x * 64;
     if (k0 >= padded) return;
-    const int vs = vt_start(p, b);
+    const long long vs = vt_start(p, b);
+    if (vs + padded > vt_cols) return;
     // load 64 keys x 128 bytes (16 bytes per thread per pass)
     for (int idx = threadIdx.x; idx < 64 * (kD / 16); idx += 256) {
         const int r = idx / (kD / 16), c = idx % (kD / 16);

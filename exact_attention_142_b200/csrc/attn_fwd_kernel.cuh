@@ -81,12 +81,13 @@ enum : int { kPairHeads = 0, kPairRows = 1 };
 
 // 2^x for a pair of arguments x <= 8 on the FMA/ALU pipes:
 // n = rint(x) via the 1.5 * 2^23 rounding constant, f = x - n in [-1/2, 1/2]
-// (exact), 2^f by the fitted cubic, and n added to the exponent bits.
-// Arguments below -125 are clamped (their weight becomes ~2^-125, far below
-// the fp32 resolution of any row sum, which is >= 1).
+// (exact), 2^f by the fitted cubic, times 2^n built in the exponent field.
+// Arguments are clamped below at -127, where the bits of 2^n, (n + 127) << 23,
+// are all zero: the result is exactly 0 for x < -126.5, and in particular for
+// -inf, so a masked key weighs exactly 0 here as it does on the MUFU path.
 __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    const uint64_t x = ptx::f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t x = ptx::f2_pack(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
     const uint64_t t = ptx::fadd2(x, ptx::f2_pack(kRound, kRound));
     const uint64_t n = ptx::fadd2(t, ptx::f2_pack(-kRound, -kRound));
     const uint64_t f = ptx::ffma2(n, ptx::f2_pack(-1.0f, -1.0f), x);
@@ -94,12 +95,13 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, fl
                             ptx::f2_pack(exp2poly::kC2, exp2poly::kC2));
     p = ptx::ffma2(p, f, ptx::f2_pack(exp2poly::kC1, exp2poly::kC1));
     p = ptx::ffma2(p, f, ptx::f2_pack(1.0f, 1.0f));
-    float p0, p1, t0, t1;
-    ptx::f2_unpack(p, p0, p1);
+    float t0, t1;
     ptx::f2_unpack(t, t0, t1);
-    // the low bits of t hold n; shifted by 23 they are n in the exponent field
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    // the low bits of t hold n; shifted by 23 they are n in the exponent field,
+    // and adding the bits of 1.0f biases it: the bits of 2^n (0 for n = -127)
+    const float s0 = __int_as_float((__float_as_int(t0) << 23) + 0x3f800000);
+    const float s1 = __int_as_float((__float_as_int(t1) << 23) + 0x3f800000);
+    ptx::f2_unpack(ptx::fmul2(p, ptx::f2_pack(s0, s1)), y0, y1);
 }
 
 struct FwdParams {
@@ -236,6 +238,7 @@ struct TilePair {
     int r0[2];
     int lo[2], hi[2];  // key-block range [lo, hi); empty when the tile is inactive
     bool active[2];
+    bool bad;          // packed boundaries inconsistent with the launch (pair skipped)
     int ulo, uhi;      // union of the two ranges
 };
 
@@ -262,9 +265,17 @@ __device__ __forceinline__ TilePair decode_pair(int u, const FwdParams& p) {
         t[0] = 2 * tp;
         t[1] = 2 * tp + 1;
     }
+    w.bad = false;
     if (p.cu_seqlens) {
-        w.start = p.cu_seqlens[w.b];
-        w.len = p.cu_seqlens[w.b + 1] - w.start;
+        // The boundaries must lie inside [0, N], must not decrease, and the
+        // sequence must fit the row blocks the launch was sized for
+        // (max_seqlen).  Otherwise the pair has no rows: nothing of it is read
+        // or written, and the producer reports the inconsistency.
+        const int s0 = p.cu_seqlens[w.b];
+        const int s1 = p.cu_seqlens[w.b + 1];
+        w.bad = s0 < 0 || s1 < s0 || s1 > p.N || (long long)(s1 - s0) > (long long)p.n_row_blocks * kBM;
+        w.start = w.bad ? 0 : s0;
+        w.len = w.bad ? 0 : s1 - s0;
     } else {
         w.start = w.b * p.N;
         w.len = p.N;
@@ -303,7 +314,8 @@ __device__ __forceinline__ bool tile_active_at(const TilePair& w, int x, int j) 
 // producer has issued every load of a pair it takes the next pending pair by
 // cancelling the launch of a CTA that has not started (cluster launch
 // control), skipping pairs with no rows (packed sequences shorter than the
-// longest), and passes it to the MMA and softmax warps through a two-entry
+// longest, and sequences whose boundaries do not fit the launch, which it
+// reports in the status word), and passes it to the MMA and softmax warps through a two-entry
 // queue in shared memory.  Pairs are thus handed out greedily in the same
 // order as by the hardware's block scheduler, while the next pair's Q load
 // and first products overlap the previous pair's epilogue.
@@ -331,6 +343,7 @@ struct UnitSource {
                 const TilePair w = decode_pair(cand, p);
                 const int u = cand;
                 cand = -1;
+                if (w.bad && (threadIdx.x & 31) == 0) atomicCAS(&g_attn_status, 0, ATTN_ERR_SEQLENS);
                 if (w.active[0] || w.active[1]) return u;
             }
             if (!more) return -1;

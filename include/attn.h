@@ -54,8 +54,12 @@ enum attn_status {
     ATTN_ERR_WORKSPACE = -8,     /* attn_fwd_host: workspace missing or too small     */
     ATTN_ERR_DEVICE_TIMEOUT = -9, /* reported by attn_device_status(): a kernel wait
                                      ran past its time limit and the kernel gave up  */
-    ATTN_ERR_PAGE = -10          /* reported by attn_device_status(): attn_decode met a
+    ATTN_ERR_PAGE = -10,         /* reported by attn_device_status(): attn_decode met a
                                     page-table entry outside [0, num_pages)          */
+    ATTN_ERR_SEQLENS = -11       /* reported by attn_device_status(): a packed batch's
+                                    cu_seqlens do not fit the call (a boundary outside
+                                    [0, N] or decreasing, or a sequence longer than
+                                    max_seqlen); that sequence was skipped            */
 };
 
 /*
@@ -71,7 +75,11 @@ enum attn_status {
  *   q   [N, Hq,  d] bf16         k, v [N, Hkv, d] bf16
  *   o   [N, Hq,  d] bf16         lse  [Hq, N] fp32
  *   max_seqlen >= the longest sequence (used only to size the launch).  The
- *   host never reads cu_seqlens; its contents are the caller's responsibility.
+ *   host never reads cu_seqlens.  The kernel checks each sequence's
+ *   boundaries before it reads or writes anything of it: a boundary outside
+ *   [0, N], a decreasing pair, or a sequence longer than max_seqlen (rounded
+ *   up to 128 rows) is skipped -- its rows of o and lse are left as they were
+ *   -- and attn_device_status() then reports ATTN_ERR_SEQLENS.
  * All tensors are contiguous (row-major in the order shown).
  *   d: head dimension, 64 or 128.
  *   scale: finite, > 0 (pass 1/sqrt(d) for the usual scaling).
@@ -243,7 +251,8 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
  * fixed device array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES (8 MiB) inside the
  * library, per device; a call whose attn_decode_workspace_bytes(...) exceeds
  * that returns ATTN_ERR_WORKSPACE before doing anything (use fewer slices, or
- * attn_decode with a workspace).  A single slice uses no scratch at all.
+ * attn_decode with a workspace).  Every argument is checked as attn_decode
+ * checks it before the array is touched.  A single slice uses no scratch.
  *
  * The first call on a device that needs the scratch looks up the array's
  * address (cudaGetSymbolAddress, with that device current) and keeps it; make
@@ -253,6 +262,11 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
  * host threads -- race on it, so order them on one stream.
  */
 #define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/* The size of that array as the library was built (ATTN_DECODE_NOALLOC_SCRATCH_BYTES):
+ * bindings read it here instead of copying the constant.  Host arithmetic only. */
+size_t attn_decode_noalloc_scratch_bytes(void);
+
 int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
                         float* lse, const int32_t* cache_seqlens, const int32_t* block_table,
                         int B, int Hq, int Hkv, int Nq, int d, int page_size, int pages_per_seq,
@@ -278,8 +292,10 @@ const char* attn_status_string(int status);
  * Call after synchronising the streams that ran attn_fwd / attn_decode.
  * Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT if any kernel since the last call
  * gave up on a bounded wait, ATTN_ERR_PAGE if attn_decode met a page-table
- * entry outside the cache (the outputs of that call are then undefined), or
- * ATTN_ERR_CUDA if a word could not be read.
+ * entry outside the cache (the outputs of that call are then undefined),
+ * ATTN_ERR_SEQLENS if a packed call's cu_seqlens did not fit its N or
+ * max_seqlen (the sequences concerned were skipped), or ATTN_ERR_CUDA if a
+ * word could not be read.
  */
 int attn_device_status(void);
 
@@ -291,6 +307,21 @@ int attn_device_status(void);
  * The GPU is never faulted or hung.  Returns the launch status.
  */
 int attn_selftest_bounded_wait(uint64_t limit_ns, struct CUstream_st* stream);
+
+/*
+ * attn_selftest_exp2_poly -- evaluates on the GPU the exponential that the
+ * forward kernels take from the FMA pipe for part of the softmax weights
+ * 2^(s - m) ("FlashAttention" explainer page, How it works, Step 3): with
+ * n = rint(x) and f = x - n in [-1/2, 1/2], 2^f from a cubic fitted for
+ * minimax relative error (csrc/gen_exp2_poly.py) times 2^n.
+ *   x, y: device float[n], 4-byte aligned; y[i] = 2^x[i] for x[i] <= 8 (the
+ *   kernels never pass more).  Relative error <= exp2poly::kMaxRelError (plus
+ *   fp32 rounding) where 2^x is a normal fp32 number, exact powers of two at
+ *   integer x, and exactly 0 for x < -126.5 and for x = -inf (a masked key).
+ * Asynchronous on `stream`.  Returns ATTN_OK, ATTN_ERR_SHAPE (n < 0),
+ * ATTN_ERR_NULL, ATTN_ERR_ALIGN, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA.
+ */
+int attn_selftest_exp2_poly(const float* x, float* y, long long n, struct CUstream_st* stream);
 
 #ifdef __cplusplus
 }

@@ -1,9 +1,16 @@
 """The C ABI library loads, exports every symbol include/attn.h declares, and
-its host-side validation returns the documented codes (no GPU needed: these
-calls return before any CUDA call)."""
+its host-side validation returns the documented codes.
+
+Every call that passes made-up device addresses runs in a child process that
+sees no GPU (CUDA_VISIBLE_DEVICES is empty): the checks under test return before
+any CUDA call, and if one of them ever regressed the call could only fail to
+find a device -- it can never launch a kernel on those addresses."""
 import ctypes
+import json
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -37,24 +44,42 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, -11, -1):
+    for code in range(0, -12, -1):
         s = ea.attn_status_string(code)
         assert s and s != "unknown status", code
     assert ea.attn_status_string(-1234) == "unknown status"
 
 
-FAKE = 1 << 20  # a 16-byte aligned fake address; validation rejects before use
+FAKE = 1 << 20  # a 16-byte aligned made-up address, only ever passed with no GPU visible
+
+_CHILD = r"""
+import json, sys
+sys.path.insert(0, sys.argv[1])
+from exact_attention_142_b200 import _binding as b
+calls = json.loads(sys.stdin.read())
+print(json.dumps([getattr(b, fn)(check=False, **kw) for fn, kw in calls]))
+"""
 
 
-def call(**over):
+def run_without_gpu(calls):
+    """[(binding function, kwargs)] -> return codes, from a child process in
+    which no GPU is visible."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    res = subprocess.run([sys.executable, "-c", _CHILD, ROOT], input=json.dumps(calls),
+                         capture_output=True, text=True, env=env, timeout=120)
+    assert res.returncode == 0, res.stderr
+    return json.loads(res.stdout.strip().splitlines()[-1])
+
+
+def fwd_args(**over):
     args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, N=16, d=128,
                 scale=0.1, causal=1, window_left=-1, window_right=-1, cu_seqlens=None,
                 max_seqlen=0, stream=0)
     args.update(over)
-    return ea.attn_fwd(check=False, **args)
+    return args
 
 
-@pytest.mark.parametrize("over,code", [
+FWD_CASES = [
     (dict(B=0), ea.ATTN_ERR_SHAPE),
     (dict(Hq=0), ea.ATTN_ERR_SHAPE),
     (dict(Hkv=0), ea.ATTN_ERR_SHAPE),
@@ -77,47 +102,19 @@ def call(**over):
     (dict(cu_seqlens=FAKE, N=10, max_seqlen=0), ea.ATTN_ERR_SHAPE),
     (dict(N=0), ea.ATTN_OK),                      # nothing to do, nothing enqueued
     (dict(N=0, q=None, k=None, v=None, o=None, lse=None), ea.ATTN_OK),
-])
-def test_validation_codes(lib, over, code):
-    assert call(**over) == code
+]
 
 
-def test_host_workspace_size(lib):
-    B, Hq, Hkv, N, d = 2, 8, 2, 100, 64
-    got = ea.attn_fwd_host_workspace_bytes(B, Hq, Hkv, N, d, False)
-    r = lambda x: (x + 255) // 256 * 256
-    tokens = B * N
-    want = r(tokens * Hq * d * 2) * 2 + 2 * r(tokens * Hkv * d * 2) + r(tokens * Hq * 4)
-    assert got == want
-    assert ea.attn_fwd_host_workspace_bytes(3, Hq, Hkv, 300, d, True) == \
-        2 * r(300 * Hq * d * 2) + 2 * r(300 * Hkv * d * 2) + r(300 * Hq * 4) + r(4 * 4)
-    assert ea.attn_fwd_host_workspace_bytes(0, Hq, Hkv, N, d, False) == 0
-
-
-def test_host_entry_rejects_missing_workspace(lib):
-    rc = ea.attn_fwd_host(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 16, 64, 0.1, True, -1, -1,
-                          None, 0, None, 0, stream=0, check=False)
-    assert rc == ea.ATTN_ERR_WORKSPACE
-
-
-def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
-    from exact_attention_142_b200 import _binding
-    monkeypatch.setattr(_binding, "_lib", None)
-    monkeypatch.setattr(_binding, "_LIB_PATH", str(tmp_path / "missing.so"))
-    with pytest.raises(RuntimeError, match="no fallback"):
-        _binding.load_library()
-
-
-def call_decode(**over):
+def call_decode_args(**over):
     args = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, o=FAKE, lse=FAKE, cache_seqlens=FAKE,
                 block_table=None, B=2, Hq=8, Hkv=2, Nq=1, d=128, page_size=16, pages_per_seq=8,
                 num_pages=16, scale=0.1, causal=1, window_left=-1, window_right=-1, num_splits=1,
                 workspace=None, workspace_bytes=0, stream=0)
     args.update(over)
-    return ea.attn_decode(check=False, **args)
+    return args
 
 
-@pytest.mark.parametrize("over,code", [
+DECODE_CASES = [
     (dict(B=0), ea.ATTN_ERR_SHAPE),
     (dict(Nq=0), ea.ATTN_ERR_SHAPE),
     (dict(Hq=6, Hkv=4), ea.ATTN_ERR_SHAPE),
@@ -139,9 +136,76 @@ def call_decode(**over):
     (dict(num_splits=4), ea.ATTN_ERR_WORKSPACE),          # 128 keys -> 2 slices, no workspace
     (dict(num_splits=4, workspace=FAKE, workspace_bytes=16), ea.ATTN_ERR_WORKSPACE),
     (dict(num_splits=4, workspace=FAKE + 16, workspace_bytes=1 << 20), ea.ATTN_ERR_WORKSPACE),
-])
-def test_decode_validation_codes(lib, over, code):
-    assert call_decode(**over) == code
+]
+
+
+def _noalloc_args(**over):
+    args = call_decode_args(**over)
+    del args["workspace"], args["workspace_bytes"]
+    return args
+
+
+# attn_decode_noalloc: attn_decode's checks, then the size of its fixed array
+# (256 sequences x 32 heads x 128 columns x 16 slices of fp32 partials: 64 MiB).
+BIG = dict(B=256, Hq=32, Hkv=8, Nq=1, d=128, page_size=64, pages_per_seq=128, num_pages=256 * 128,
+           num_splits=16)
+NOALLOC_CASES = [
+    (dict(BIG), ea.ATTN_ERR_WORKSPACE),
+    (dict(BIG, q=None), ea.ATTN_ERR_NULL),
+    (dict(BIG, d=80), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(num_splits=0), ea.ATTN_ERR_SHAPE),
+]
+
+HOST_CASES = [
+    (dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=16, d=64, scale=0.1,
+          causal=True, window_left=-1, window_right=-1, cu_seqlens=None, max_seqlen=0,
+          workspace=None, workspace_bytes=0, stream=0), ea.ATTN_ERR_WORKSPACE),
+]
+
+_ALL = ([("attn_fwd", fwd_args(**o), c) for o, c in FWD_CASES] +
+        [("attn_decode", call_decode_args(**o), c) for o, c in DECODE_CASES] +
+        [("attn_decode_noalloc", _noalloc_args(**o), c) for o, c in NOALLOC_CASES] +
+        [("attn_fwd_host", kw, c) for kw, c in HOST_CASES])
+
+
+@pytest.fixture(scope="module")
+def no_gpu_codes(lib):
+    return run_without_gpu([(fn, kw) for fn, kw, _ in _ALL])
+
+
+@pytest.mark.parametrize("idx", range(len(_ALL)),
+                         ids=[f"{fn}-{i}" for i, (fn, _, _) in enumerate(_ALL)])
+def test_validation_codes(no_gpu_codes, idx):
+    fn, kw, code = _ALL[idx]
+    assert no_gpu_codes[idx] == code, (fn, kw)
+
+
+def test_noalloc_scratch_size_matches_header(lib):
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    m = re.search(r"#define\s+ATTN_DECODE_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*\*\s*1024u\s*\*\s*1024u\)",
+                  text)
+    assert m, "ATTN_DECODE_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert ea.attn_decode_noalloc_scratch_bytes() == int(m.group(1)) * 1024 * 1024
+
+
+def test_host_workspace_size(lib):
+    B, Hq, Hkv, N, d = 2, 8, 2, 100, 64
+    got = ea.attn_fwd_host_workspace_bytes(B, Hq, Hkv, N, d, False)
+    r = lambda x: (x + 255) // 256 * 256
+    tokens = B * N
+    want = r(tokens * Hq * d * 2) * 2 + 2 * r(tokens * Hkv * d * 2) + r(tokens * Hq * 4)
+    assert got == want
+    assert ea.attn_fwd_host_workspace_bytes(3, Hq, Hkv, 300, d, True) == \
+        2 * r(300 * Hq * d * 2) + 2 * r(300 * Hkv * d * 2) + r(300 * Hq * 4) + r(4 * 4)
+    assert ea.attn_fwd_host_workspace_bytes(0, Hq, Hkv, N, d, False) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from exact_attention_142_b200 import _binding
+    monkeypatch.setattr(_binding, "_lib", None)
+    monkeypatch.setattr(_binding, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        _binding.load_library()
 
 
 def test_decode_workspace_size(lib):

@@ -349,3 +349,114 @@ def test_attention_convenience_dense_and_packed():
     o_ref, lse_ref, _ = oracle_run(q, k, v, B=len(lengths), Hq=Hq, Hkv=Hkv, N=T, d=d,
                                    scale=default_scale(d), causal=True, cu_seqlens=cu)
     compare_full(o.cpu(), lse.cpu(), o_ref, lse_ref)
+
+
+# A key that the mask hides must weigh exactly 0 ("FlashAttention" explainer
+# page, "Checking correctness": the reference fills masked scores with -inf).
+# V is set to 1e37 (finite in bf16) on chosen keys; a row that sees none of them
+# must still match the oracle, which fails if a hidden key kept any weight
+# above ~1e-39 (a weight of 2^-125 would add ~0.2 to O).  The chosen keys sit in
+# the columns 28-31 of every 32 of a key block, where the kernels take some
+# exponentials from the FMA pipe, and past the end of a packed sequence.  Q is
+# scaled up so that one key dominates each row and the row sum stays near 1.
+HUGE_V = 1e37
+
+
+def _huge_masked_probe(lengths, Hq, Hkv, d, causal, left, right, packed, huge, seed):
+    B = len(lengths)
+    if packed:
+        cu = W.cumulative(lengths)
+        N = T = cu[-1]
+        shape_q, shape_kv = (T, Hq, d), (T, Hkv, d)
+        tok = lambda b, j: cu[b] + j  # noqa: E731
+    else:
+        cu = None
+        N = lengths[0]
+        T = B * N
+        shape_q, shape_kv = (B, N, Hq, d), (B, N, Hkv, d)
+        tok = lambda b, j: b * N + j  # noqa: E731
+    q, k, v = W.draw_qkv(shape_q, shape_kv, seed)
+    q = (q.float() * 4).to(torch.bfloat16)
+    vf = v.reshape(T, Hkv, d).clone()
+    hidden = {b: np.array([j for j in range(L) if huge(b, j)], dtype=np.int64)
+              for b, L in enumerate(lengths)}
+    for b, js in hidden.items():
+        for j in js:
+            vf[tok(b, int(j))] = HUGE_V
+    v = vf.reshape(shape_kv).contiguous()
+    kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=causal,
+              window_left=left, window_right=right, cu_seqlens=cu)
+    o, lse = gpu_run(q, k, v, **kw)
+    r = 0 if causal else right
+    rows, sensitive = [], 0
+    for b, L in enumerate(lengths):
+        js = hidden[b]
+        for i in range(L):
+            lo = 0 if left < 0 else max(0, i - left)
+            hi = L - 1 if r < 0 else min(L - 1, i + r)
+            if np.any((js >= lo) & (js <= hi)):
+                continue  # this row sees a huge value
+            # the key blocks the row's tile reads (128-key blocks from the
+            # sequence start) hold a hidden huge key, or the next sequence does
+            blk_lo, blk_hi = lo // 128 * 128, (hi // 128 + 1) * 128
+            if np.any((js >= blk_lo) & (js < blk_hi)) or (packed and blk_hi > L and b + 1 < B and
+                                                           hidden[b + 1].size):
+                sensitive += 1
+            for h in range(Hq):
+                rows.append((b, h, i))
+    assert sensitive > 0
+    rows = np.array(rows, dtype=np.int64)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, rows=rows, **kw)
+    of = o.reshape(-1, Hq, d)
+    lf = lse.reshape(-1)
+    got_o = np.stack([of[o_index(cu, b, i, N), h].to(torch.float64).numpy() for b, h, i in rows])
+    got_l = np.array([float(lf[lse_index(cu, b, h, i, Hq, N)]) for b, h, i in rows])
+    assert np.isfinite(got_o).all()
+    assert np.abs(got_o - o_ref).max() <= TOL_O, np.abs(got_o - o_ref).max()
+    assert np.abs(got_l - lse_ref).max() <= TOL_LSE
+
+
+@pytest.mark.parametrize("probe", [
+    # name, lengths, Hq, Hkv, d, causal, left, right, packed, huge(b, j)
+    ("causal_diagonal_block", [384, 384], 2, 2, 128, True, -1, -1, False,
+     lambda b, j: j % 128 >= 92 and j % 32 >= 28),
+    ("window_left_causal", [700], 4, 2, 128, True, 16, 0, False, lambda b, j: j % 32 >= 28),
+    ("window_two_sided_d64", [600], 2, 1, 64, False, 8, 8, False, lambda b, j: j % 32 >= 28),
+    ("packed_neighbour_noncausal", [200, 300, 150], 2, 2, 128, False, -1, -1, True,
+     lambda b, j: b == 1),
+    ("packed_neighbour_causal_gqa", [200, 300, 150], 4, 2, 128, True, -1, -1, True,
+     lambda b, j: b == 1),
+], ids=lambda p: p[0])
+def test_masked_keys_weigh_exactly_zero(probe):
+    _, lengths, Hq, Hkv, d, causal, left, right, packed, huge = probe
+    _huge_masked_probe(lengths, Hq, Hkv, d, causal, left, right, packed, huge, seed=71)
+
+
+def test_packed_max_seqlen_too_small_is_reported():
+    """A sequence longer than max_seqlen (rounded up to 128 rows) does not fit
+    the launch: it is skipped -- its rows are left as they were -- and the
+    status word reports it; the other sequences are computed, and the next call
+    is clean.  Every address stays inside the tensors."""
+    lengths = [300, 129, 50]
+    cu = W.cumulative(lengths)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 128
+    q, k, v = W.draw_qkv((T, Hq, d), (T, Hkv, d), 72)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    cud = torch.tensor(cu, dtype=torch.int32, device=dev)
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full((Hq, T), float("nan"), dtype=torch.float32, device=dev)
+    assert ea.attn_device_status() == ea.ATTN_OK
+    ea.attn_fwd(qd, kd, vd, o, lse, 3, Hq, Hkv, T, d, default_scale(d), True, -1, -1, cud, 200)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_ERR_SEQLENS
+    assert ea.attn_device_status() == ea.ATTN_OK  # read clears it
+    o, lse = o.cpu(), lse.cpu()
+    assert torch.isnan(o[:300].float()).all() and torch.isnan(lse[:, :300]).all()
+    kw = dict(B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=default_scale(d), causal=True, cu_seqlens=cu)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    o_ref = o_ref.reshape(T, Hq, d)
+    assert np.abs(o[300:].double().numpy() - o_ref[300:]).max() <= TOL_O
+    assert np.abs(lse[:, 300:].double().numpy() - lse_ref.reshape(Hq, T)[:, 300:]).max() <= TOL_LSE
+    o2, lse2 = gpu_run(q, k, v, max_seqlen=300, **kw)  # asserts a clean status
+    compare_full(o2, lse2, o_ref, lse_ref)

@@ -146,3 +146,35 @@ def test_bwd_causal_gqa_workload_one_group():
     ref = ref_bwd(subq(q), subk(k), subk(v), subq(do), B=1, Hq=grp, Hkv=1, N=w.N, d=w.d,
                   scale=w.scale, causal=True)
     compare((dq[b:b + 1, :, hs], dk[b:b + 1, :, gkv:gkv + 1], dv[b:b + 1, :, gkv:gkv + 1]), ref)
+
+
+def test_bwd_packed_max_seqlen_too_small_is_reported():
+    """A sequence longer than max_seqlen (rounded up to 128) is skipped by the
+    gradient kernels -- its rows of dq, dk, dv are left as they were -- and the
+    status word reports it; the other sequences match a call with the right
+    max_seqlen.  Every address stays inside the tensors."""
+    lens = [300, 129, 50]
+    cu = W.cumulative(lens)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 128
+    q, k, v, do = draw((T, Hq, d), (T, Hkv, d), 81)
+    scale = default_scale(d)
+    good = gpu_bwd(q, k, v, do, B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=scale, causal=True, cu=cu)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    cud = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    o = torch.empty_like(qd)
+    lse = torch.empty((Hq * T,), dtype=torch.float32, device=DEV)
+    ea.attn_fwd(qd, kd, vd, o, lse, 3, Hq, Hkv, T, d, scale, True, -1, -1, cud, 300)
+    dq = torch.full_like(qd, float("nan"))
+    dk = torch.full_like(kd, float("nan"))
+    dv = torch.full_like(vd, float("nan"))
+    nbytes = ea.attn_bwd_workspace_bytes(3, Hq, Hkv, T, d, True)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=DEV)
+    ea.attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, 3, Hq, Hkv, T, d, scale, True, -1, -1, cud, 200,
+                ws, nbytes)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_ERR_SEQLENS
+    assert ea.attn_device_status() == ea.ATTN_OK
+    for got, ref in zip((dq.cpu(), dk.cpu(), dv.cpu()), good):
+        assert torch.isnan(got[:300].float()).all()
+        g, r = got[300:].double(), ref[300:].double()
+        assert float((g - r).abs().max()) <= REL_TOL * float(r.abs().max()) + ABS_FLOOR

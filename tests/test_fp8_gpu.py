@@ -224,3 +224,30 @@ def test_fp8_schedule_many_pairs_per_cta():
                -1, -1, [N] * B, Hq // Hkv)
     # every row of every pair was written
     assert np.isfinite(og).all() and np.isfinite(lg).all()
+
+
+def test_fp8_packed_max_seqlen_too_small_is_reported():
+    """As attn_fwd: a sequence longer than max_seqlen (rounded up to 128 rows)
+    is skipped, nothing of it is read or written, and the status word reports
+    it; the other sequences equal a call with the right max_seqlen."""
+    lens = [300, 129, 50]
+    cu = W.cumulative(lens)
+    T, Hq, Hkv, d = cu[-1], 4, 2, 128
+    q, k, v = W.draw_qkv_e4m3((T, Hq, d), (T, Hkv, d), seed=18)
+    scale = default_scale(d)
+    good_o, good_l = gpu_fp8(q, k, v, B=3, Hq=Hq, Hkv=Hkv, N=T, d=d, scale=scale, causal=True,
+                             cu=cu)
+    qd, kd, vd = (t.view(torch.uint8).to(DEV) for t in (q, k, v))
+    cud = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    o = torch.full((T, Hq, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((Hq, T), float("nan"), dtype=torch.float32, device=DEV)
+    nbytes = ea.attn_fwd_fp8_workspace_bytes(3, Hq, Hkv, T, d, True)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    ea.attn_fwd_fp8(qd, kd, vd, o, lse, 3, Hq, Hkv, T, d, scale, True, -1, -1, cud, 200, ws, nbytes)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_ERR_SEQLENS
+    assert ea.attn_device_status() == ea.ATTN_OK
+    o, lse = o.cpu(), lse.cpu()
+    assert torch.isnan(o[:300].float()).all() and torch.isnan(lse[:, :300]).all()
+    assert torch.equal(o[300:], good_o[300:])
+    assert torch.equal(lse[:, 300:], good_l.reshape(Hq, T)[:, 300:])
