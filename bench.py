@@ -16,10 +16,18 @@ launching stream; L2 is flushed between timed steps (outside the events).
 (attn_fwd_host) with pinned host buffers: host->device copies of q, k, v, the
 kernel and device->host copies of o and lse are all inside the timed region.
 
-With N > 1 (torchrun, one process per GPU) every rank runs the same workload on
-its own GPU (independent replicas, weak scaling); the time is the max over
-ranks and the value is all ranks' FLOPs over that time.  There is no
-collective on the data path.
+With N > 1 (torchrun, one process per GPU) every rank runs one batch shard of
+the workload's size on its own GPU (weak scaling: the global batch is N times
+the workload's); the time is the max over ranks and the value is all ranks'
+FLOPs over that time.  --split heads|sequences|auto instead splits ONE
+workload over the ranks (strong scaling; exact_attention_142_b200/split.py):
+whole GQA groups of heads, or contiguous sequence ranges balanced by their
+visible pairs.  There is no collective on the data path either way.
+
+The default run (workload 3) also times the other d = 128 workloads (2, 4, 5)
+the same way ("other_workloads") and runs the headline workload back to back
+for about 2.5 s with the SM clock sampled ("sustained"), to hold against the
+sustained matmul peak; --no-extra skips both.
 
 --impl reference times the CPU oracle (fp64, all host cores) on bounded
 samples of the same workload (rank 0 only).
@@ -311,6 +319,103 @@ def run_cuda(args, w: W.Workload, rank: int, world: int, local_rank: int):
         kernel_ms, e2e_ms = float(t[0]), float(t[1])
     run_cuda.step_times = sorted(times)
     return kernel_ms, e2e_ms, h2d, d2h, clocks
+
+
+def time_forward(w: W.Workload, dev, steps: int, warmup: int, flush=None):
+    """attn_fwd on one workload, timed like the benchmark's steps (L2 flushed
+    between calls, outside the events): the per-call times in ms."""
+    import torch
+
+    import exact_attention_142_b200 as ea
+    q, k, v = W.inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    del q, k, v
+    o = torch.empty_like(qd)
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=dev) if w.packed else None
+    lse = torch.empty((w.Hq, w.tokens) if w.packed else (w.B, w.Hq, w.N), dtype=torch.float32,
+                      device=dev)
+    if flush is None:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: ea.attn_fwd(qd, kd, vd, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale,  # noqa: E731
+                               w.causal, w.window_left, w.window_right, cu, w.max_seqlen, stream)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError(f"device status reported an error on {w.name}")
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def other_workloads(dev, steps: int, warmup: int, peak: float):
+    """The other d = 128 workloads, each timed like the headline one."""
+    out = {}
+    for cfg in (2, 4, 5):
+        w = W.workload(cfg)
+        times = time_forward(w, dev, steps, warmup)
+        ms = sum(times) / len(times)
+        tf = flops_of(w) / (ms * 1e-3) / 1e12
+        out[w.name] = {"ms_per_step": ms, "steps": steps, "value": tf, "unit": UNIT,
+                       "frac": tf / peak, "frac_of_spec_2250": tf / SPEC_BF16_TFLOPS,
+                       "step_ms": step_stats(times), "flop_per_step": flops_of(w),
+                       "gpu_launches": steps, "l2": "flushed between timed steps"}
+    return out
+
+
+def sustained_forward(w: W.Workload, dev, seconds: float, peak_sustained: float):
+    """Back-to-back calls (no flush; the inputs, 2x the L2, stream through it)
+    for at least `seconds`, under the power cap, with the SM clock sampled
+    over the loop: the figure to hold against the sustained matmul peak."""
+    import torch
+
+    import exact_attention_142_b200 as ea
+    q, k, v = W.inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    del q, k, v
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: ea.attn_fwd(qd, kd, vd, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale,  # noqa: E731
+                               w.causal, w.window_left, w.window_right, None, 0, stream)
+    for _ in range(5):
+        call()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(10):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    n = max(20, int(seconds / (a.elapsed_time(b) / 10 * 1e-3)))
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    sampler.mark_begin()
+    a.record(stream)
+    for _ in range(n):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark_end()
+    clocks = sampler.stop()
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported an error in the sustained loop")
+    ms = a.elapsed_time(b) / n
+    tf = flops_of(w) / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "value": tf, "unit": UNIT, "ms_per_step": ms, "steps": n,
+            "seconds": ms * n * 1e-3, "gpu_launches": n,
+            "frac_of_sustained": (tf / peak_sustained) if peak_sustained else None,
+            "peak_sustained": peak_sustained, "frac_of_spec_2250": tf / SPEC_BF16_TFLOPS,
+            "clocks": clocks, "l2": "not flushed (back-to-back calls; inputs 2.7x L2)"}
 
 
 # ---------------------------------------------------------------------------
@@ -1180,13 +1285,114 @@ def main_fp8(args, w: W.Workload, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def config_dict(w: W.Workload, n_gpus: int):
+def config_dict(w: W.Workload, n_gpus: int, split_mode: str = "none"):
+    par = (f"one batch shard per rank x{n_gpus} (no collective)" if split_mode == "none"
+           else f"{split_mode} split of one workload over {n_gpus} ranks (no collective)")
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "N": w.N if not w.packed else None, "tokens": w.tokens, "d": w.d,
             "causal": w.causal, "window": [w.window_left, w.window_right],
             "packed_sequences": len(w.cu_seqlens) - 1 if w.packed else None,
             "flop_per_step": flops_of(w), "l2": "flushed between timed steps",
-            "parallelism": f"replicas x{n_gpus} (no collective)"}
+            "parallelism": par}
+
+
+def main_split(args, w: W.Workload, rank, world, local_rank):
+    """One workload split over the ranks (heads or sequences): each rank runs
+    attn_fwd on its shard; the time is the slowest rank's, the value the whole
+    workload's FLOPs over it (strong scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_142_b200 as ea
+    from exact_attention_142_b200 import split
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ea.load_library()
+    lengths = ([b - a for a, b in zip(w.cu_seqlens[:-1], w.cu_seqlens[1:])] if w.packed
+               else [w.N] * w.B)
+    shards = split.plan(world, args.split, B=w.B, Hq=w.Hq, Hkv=w.Hkv, lengths=lengths,
+                        causal=w.causal, left=w.window_left, right=w.window_right)
+    sh = shards[rank]
+    q, k, v = W.inputs(w)
+    qs, ks, vs, cu, B, Hq, Hkv = split.shard_inputs(q, k, v, sh, w.cu_seqlens if w.packed else None)
+    del q, k, v
+    my_flops = 0.0
+    if not sh.empty:
+        my_lengths = lengths[sh.seqs[0]:sh.seqs[1]]
+        my_flops = 4.0 * w.d * Hq * sum(split.visible_pairs(L, w.causal, w.window_left,
+                                                            w.window_right) for L in my_lengths)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    times = [0.0] * args.steps
+    if not sh.empty:
+        qd, kd, vd = qs.to(dev), ks.to(dev), vs.to(dev)
+        N = qd.shape[0] if cu is not None else w.N
+        o = torch.empty_like(qd)
+        lse = torch.empty((Hq, N) if cu is not None else (B, Hq, N), dtype=torch.float32, device=dev)
+        cud = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
+        max_len = max(lengths[sh.seqs[0]:sh.seqs[1]])
+
+        def step():
+            ea.attn_fwd(qd, kd, vd, o, lse, B, Hq, Hkv, N, w.d, w.scale, w.causal, w.window_left,
+                        w.window_right, cud, max_len, stream)
+    else:
+        def step():
+            pass
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.mark_end()
+    times = [a.elapsed_time(b) for a, b in ev]
+    if ea.attn_device_status() != ea.ATTN_OK:
+        raise RuntimeError("device status reported an error during the timed region")
+    ms = sum(times) / len(times)
+    clocks = sampler.stop() if sampler else None
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t[0])
+    if rank == 0:
+        fl = flops_of(w)
+        value = fl / (ms_max * 1e-3) / 1e12
+        peaks, src = measured_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal bf16 Q, K, V)",
+            "config": config_dict(w, world, args.split) | {
+                "shards": [{"rank": s.rank, "heads": list(s.heads), "kv_heads": list(s.kv_heads),
+                            "seqs": list(s.seqs)} for s in shards]},
+            "gpu_launches": args.steps,
+            "rank0": {"ms_per_step": ms, "flop_per_step": my_flops},
+            "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": UNIT,
+                         "frac": value / world / peak,
+                         "note": "per GPU: the whole workload's FLOPs / slowest rank / ranks"},
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -1209,6 +1415,12 @@ def main():
     ap.add_argument("--sdpa-backend", default="all", choices=["all", "cudnn", "flash", "efficient"],
                     help="--impl torch_sdpa only: the backends to time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other d = 128 workloads and the sustained loop (default "
+                         "workload only)")
+    ap.add_argument("--split", default="none", choices=["none", "heads", "sequences", "auto"],
+                    help="with --gpus N: split ONE workload over the ranks (strong scaling) "
+                         "instead of one batch shard per rank (weak scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -1245,8 +1457,23 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.split != "none":
+        try:
+            main_split(args, w, rank, world, local_rank)
+        finally:
+            if world > 1:
+                dist.destroy_process_group()
+        return
+    extra = sustained_run = None
     try:
         kernel_ms, e2e_ms, h2d, d2h, clocks = run_cuda(args, w, rank, world, local_rank)
+        if rank == 0 and args.workload == "3" and not args.no_extra:
+            dev = torch.device("cuda", local_rank)
+            peaks, _ = measured_peaks()
+            extra = other_workloads(dev, args.steps, args.warmup,
+                                    float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)))
+            sustained_run = sustained_forward(w, dev, 2.5,
+                                          float(peaks.get("bf16_tflops_sustained", 0.0)) or None)
     finally:
         if world > 1:
             dist.barrier()
@@ -1279,6 +1506,10 @@ def main():
             "clocks": clocks,
             "step_ms": step_stats(run_cuda.step_times),
         }
+        if extra is not None:
+            line["other_workloads"] = extra
+        if sustained_run is not None:
+            line["sustained"] = sustained_run
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

@@ -353,12 +353,12 @@ def test_attention_convenience_dense_and_packed():
 
 # A key that the mask hides must weigh exactly 0 ("FlashAttention" explainer
 # page, "Checking correctness": the reference fills masked scores with -inf).
-# V is set to 1e37 (finite in bf16) on chosen keys; a row that sees none of them
-# must still match the oracle, which fails if a hidden key kept any weight
-# above ~1e-39 (a weight of 2^-125 would add ~0.2 to O).  The chosen keys sit in
-# the columns 28-31 of every 32 of a key block, where the kernels take some
-# exponentials from the FMA pipe, and past the end of a packed sequence.  Q is
-# scaled up so that one key dominates each row and the row sum stays near 1.
+# The same call runs twice, once with V = 1e37 (finite in bf16) on chosen keys:
+# every row that sees none of them must come out bit-identical, which fails if a
+# hidden key kept any weight at all (a weight of 2^-125 would add ~0.2 to O).
+# The chosen keys sit in the columns 28-31 of every 32 of a key block, where the
+# kernels take some exponentials from the FMA pipe, and past the end of a packed
+# sequence.  The run with ordinary values is also checked against the oracle.
 HUGE_V = 1e37
 
 
@@ -376,17 +376,19 @@ def _huge_masked_probe(lengths, Hq, Hkv, d, causal, left, right, packed, huge, s
         shape_q, shape_kv = (B, N, Hq, d), (B, N, Hkv, d)
         tok = lambda b, j: b * N + j  # noqa: E731
     q, k, v = W.draw_qkv(shape_q, shape_kv, seed)
-    q = (q.float() * 4).to(torch.bfloat16)
     vf = v.reshape(T, Hkv, d).clone()
     hidden = {b: np.array([j for j in range(L) if huge(b, j)], dtype=np.int64)
               for b, L in enumerate(lengths)}
     for b, js in hidden.items():
         for j in js:
             vf[tok(b, int(j))] = HUGE_V
-    v = vf.reshape(shape_kv).contiguous()
+    v_huge = vf.reshape(shape_kv).contiguous()
     kw = dict(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, scale=default_scale(d), causal=causal,
               window_left=left, window_right=right, cu_seqlens=cu)
     o, lse = gpu_run(q, k, v, **kw)
+    o_h, lse_h = gpu_run(q, k, v_huge, **kw)
+    o_ref, lse_ref, _ = oracle_run(q, k, v, **kw)
+    compare_full(o, lse, o_ref, lse_ref)
     r = 0 if causal else right
     rows, sensitive = [], 0
     for b, L in enumerate(lengths):
@@ -402,18 +404,14 @@ def _huge_masked_probe(lengths, Hq, Hkv, d, causal, left, right, packed, huge, s
             if np.any((js >= blk_lo) & (js < blk_hi)) or (packed and blk_hi > L and b + 1 < B and
                                                            hidden[b + 1].size):
                 sensitive += 1
+            rows.append(o_index(cu, b, i, N))
             for h in range(Hq):
-                rows.append((b, h, i))
+                idx = lse_index(cu, b, h, i, Hq, N)
+                assert lse_h.reshape(-1)[idx] == lse.reshape(-1)[idx], (b, h, i)
     assert sensitive > 0
-    rows = np.array(rows, dtype=np.int64)
-    o_ref, lse_ref, _ = oracle_run(q, k, v, rows=rows, **kw)
-    of = o.reshape(-1, Hq, d)
-    lf = lse.reshape(-1)
-    got_o = np.stack([of[o_index(cu, b, i, N), h].to(torch.float64).numpy() for b, h, i in rows])
-    got_l = np.array([float(lf[lse_index(cu, b, h, i, Hq, N)]) for b, h, i in rows])
-    assert np.isfinite(got_o).all()
-    assert np.abs(got_o - o_ref).max() <= TOL_O, np.abs(got_o - o_ref).max()
-    assert np.abs(got_l - lse_ref).max() <= TOL_LSE
+    rows = torch.tensor(rows)
+    of, ohf = o.reshape(-1, Hq, d), o_h.reshape(-1, Hq, d)
+    assert torch.equal(ohf[rows], of[rows])
 
 
 @pytest.mark.parametrize("probe", [
