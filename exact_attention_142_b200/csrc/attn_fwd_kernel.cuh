@@ -540,18 +540,26 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
         f ^= kQ;
         f |= kFirst | (kFirst << 1);
         ptx::tc_fence_after_sync();
-        // Issue order per key block j:  S0(j), PV1(j-1), S1(j), PV0(j).  Each
-        // softmax group then has the two products of the other tile to hide its
-        // exponentials behind.  S_x(j) overwrites the P_x(j-1) columns only after
-        // PV_x(j-1) was issued; tcgen05 MMAs from one thread execute in order.
-        for (int j = w.ulo; ok && j < w.uhi; ++j, ring += 2) {
-            const int ks = ring % STAGES, vs = (ring + 1) % STAGES;
+        // Issue order per key block j:  PV1(j-1), S1(j), PV0(j), S0(j+1), with
+        // S0 of the pair's first block before the loop.  Each softmax group
+        // then has the two products of the other tile to hide its
+        // exponentials behind, and each tile's P V product is followed at once
+        // by its next score product: the value tile of block j and the key
+        // tile of block j+1 are awaited before the tile's weights are, so no
+        // wait sits between the two.  S_x(j) overwrites the P_x(j-1) columns
+        // only after PV_x(j-1) was issued; tcgen05 MMAs from one thread
+        // execute in order.
+        if (w.uhi > w.ulo) {
+            const int ks = ring % STAGES;
             if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (ring / STAGES) & 1, abort_flag, lim))) break;
             ptx::tc_fence_after_sync();
-            if (j >= lo0 && j < hi0) {
+            if (w.ulo >= lo0 && w.ulo < hi0) {
                 qk(0, ks);
                 ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
             }
+        }
+        for (int j = w.ulo; ok && j < w.uhi; ++j, ring += 2) {
+            const int ks = ring % STAGES, vs = (ring + 1) % STAGES, nks = (ring + 2) % STAGES;
             if (j > w.ulo) {
                 const int pvs = (ring - 1) % STAGES;
                 if (j - 1 >= lo1 && j - 1 < hi1 && !(ok = pv(1, pvs, j - 1 == hi1 - 1))) break;
@@ -563,9 +571,16 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
             }
             ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
             if (j == w.uhi - 1) ptx::tc_commit_elect(L::bar_q_empty(sbase));  // last score products issued
+            const bool more = j + 1 < w.uhi;
             if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), ((ring + 1) / STAGES) & 1, abort_flag, lim))) break;
+            if (more && !(ok = warp_wait(L::bar_kv_full(sbase, nks), ((ring + 2) / STAGES) & 1, abort_flag, lim)))
+                break;
             ptx::tc_fence_after_sync();
             if (j >= lo0 && j < hi0 && !(ok = pv(0, vs, j == hi0 - 1))) break;
+            if (more && j + 1 >= lo0 && j + 1 < hi0) {
+                qk(0, nks);
+                ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
+            }
         }
         if (!ok) break;
         if (w.uhi > w.ulo) {
