@@ -210,6 +210,90 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, uint32_t
     return ptx::smem_desc_sw128(tile + kk * 2048, box, 1024);
 }
 
+// All K-steps of one product from a single elected lane: the per-step
+// descriptors are computed by the converged warp, and one elect.sync block
+// issues the steps back to back (the first accumulates into D only if
+// `accumulate`, the others always).
+__device__ __forceinline__ void mma_ss4_elect(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %9, 0;\n\t"
+        "setp.eq.b32 t, %9, %9;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %10, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %10, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %10, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %10, t;\n\t}" ::"r"(d),
+        "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+        "r"(accumulate), "r"(idesc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts4_elect(uint32_t d, const uint32_t (&a)[4], const uint64_t (&b)[4],
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %9, 0;\n\t"
+        "setp.eq.b32 t, %9, %9;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %10, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %10, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %10, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %10, t;\n\t}" ::"r"(d),
+        "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+        "r"(accumulate), "r"(idesc)
+        : "memory");
+}
+
+// S^T / dP^T (dkv kernel): both operands K-major from shared memory, the
+// D / 16 steps of d in groups of four (the second group accumulates).
+template <int D>
+__device__ __forceinline__ void mma_ss_kmajor_d(uint32_t d, uint32_t a_tile, uint32_t a_box, uint32_t b_tile,
+                                                uint32_t b_box, uint32_t idesc) {
+#pragma unroll
+    for (int g = 0; g < D / 64; ++g) {
+        uint64_t a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[i] = kmajor_desc(a_tile, 4 * g + i, a_box);
+            b[i] = kmajor_desc(b_tile, 4 * g + i, b_box);
+        }
+        mma_ss4_elect(d, a, b, idesc, g > 0 ? 1u : 0u);
+    }
+}
+
+// S / dP (dq kernel): A from tensor memory (8 columns per step), B K-major.
+template <int D>
+__device__ __forceinline__ void mma_ts_kmajor_d(uint32_t d, uint32_t a_tmem, uint32_t b_tile, uint32_t b_box,
+                                                uint32_t idesc) {
+#pragma unroll
+    for (int g = 0; g < D / 64; ++g) {
+        uint32_t a[4];
+        uint64_t b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[i] = a_tmem + 8 * (4 * g + i);
+            b[i] = kmajor_desc(b_tile, 4 * g + i, b_box);
+        }
+        mma_ts4_elect(d, a, b, idesc, g > 0 ? 1u : 0u);
+    }
+}
+
+// Gradient products over one 64-wide step: A from tensor memory (the bf16
+// pairs of 16 rows at columns 16 kk), B MN-major.
+__device__ __forceinline__ void mma_ts_grad4(uint32_t d, uint32_t a_tmem, uint32_t b_tile, uint32_t b_box,
+                                             uint32_t idesc, uint32_t accumulate) {
+    uint32_t a[4];
+    uint64_t b[4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        a[kk] = a_tmem + 16 * kk;
+        b[kk] = mnmajor_desc(b_tile, kk, b_box);
+    }
+    mma_ts4_elect(d, a, b, idesc, accumulate);
+}
+
 // ------------------------------------------------------------ D = rowsum(dO * O)
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_dsum(const BwdParams p) {
@@ -390,14 +474,9 @@ __device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, ui
         if (!warp_wait(L::bar_full(sbase, s), (t / STAGES) & 1, abort_flag, lim)) return false;
         ptx::tc_fence_after_sync();
         const uint32_t buf = (t & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)  // S^T = K Q^T
-            ptx::mma_ss_elect(tmem + buf, kmajor_desc(sbase + L::kK, kk, kBox128),
-                              kmajor_desc(L::q(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)  // dP^T = V dO^T
-            ptx::mma_ss_elect(tmem + 128 + buf, kmajor_desc(sbase + L::kV, kk, kBox128),
-                              kmajor_desc(L::dout(sbase, s), kk, kBox64), kIdS, kk > 0 ? 1u : 0u);
+        mma_ss_kmajor_d<D>(tmem + buf, sbase + L::kK, kBox128, L::q(sbase, s), kBox64, kIdS);  // S^T = K Q^T
+        mma_ss_kmajor_d<D>(tmem + 128 + buf, sbase + L::kV, kBox128, L::dout(sbase, s), kBox64,
+                           kIdS);  // dP^T = V dO^T
         ptx::tc_commit_elect(L::bar_st(sbase, t & 1));
         return true;
     };
@@ -408,14 +487,10 @@ __device__ __forceinline__ void dkv_mma(const DkvWork& w, const BwdParams& p, ui
         ptx::tc_fence_after_sync();
         const int s = t % STAGES;
         const uint32_t buf = (t & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < kStep / 16; ++kk)  // dV += P^T dO  (P^T of queries 16kk.. at column 16kk)
-            ptx::mma_ts_elect(tmem + 256, tmem + buf + 16 * kk, mnmajor_desc(L::dout(sbase, s), kk, kBox64),
-                              kIdG, (t > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < kStep / 16; ++kk)  // dK += dS^T Q
-            ptx::mma_ts_elect(tmem + 384, tmem + 128 + buf + 16 * kk, mnmajor_desc(L::q(sbase, s), kk, kBox64),
-                              kIdG, (t > 0 || kk > 0) ? 1u : 0u);
+        static_assert(kStep == 64, "four 16-row steps per gradient product");
+        // dV += P^T dO  (P^T of queries 16kk.. at column 16kk), then dK += dS^T Q
+        mma_ts_grad4(tmem + 256, tmem + buf, L::dout(sbase, s), kBox64, kIdG, t > 0 ? 1u : 0u);
+        mma_ts_grad4(tmem + 384, tmem + 128 + buf, L::q(sbase, s), kBox64, kIdG, t > 0 ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_empty(sbase, s));
     }
     ptx::tc_commit_elect(L::bar_done(sbase));
@@ -713,14 +788,8 @@ __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint
         // A from tensor memory: shared memory then serves only the 64-key B
         // operand (an SS product of N = 64 would read 1.5x the shared-memory
         // bandwidth that the tensor pipe consumes).
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)  // S = Q K^T
-            ptx::mma_ts_elect(tmem + buf, tmem + L::kTQ + 8 * kk, kmajor_desc(L::k(sbase, s), kk, kBox64), kIdS,
-                              kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)  // dP = dO V^T
-            ptx::mma_ts_elect(tmem + 128 + buf, tmem + L::kTDO + 8 * kk, kmajor_desc(L::v(sbase, s), kk, kBox64),
-                              kIdS, kk > 0 ? 1u : 0u);
+        mma_ts_kmajor_d<D>(tmem + buf, tmem + L::kTQ, L::k(sbase, s), kBox64, kIdS);          // S = Q K^T
+        mma_ts_kmajor_d<D>(tmem + 128 + buf, tmem + L::kTDO, L::v(sbase, s), kBox64, kIdS);   // dP = dO V^T
         ptx::tc_commit_elect(L::bar_st(sbase, t & 1));
         return true;
     };
@@ -731,10 +800,8 @@ __device__ __forceinline__ void dq_mma(const DqWork& w, const BwdParams& p, uint
         ptx::tc_fence_after_sync();
         const int s = t % STAGES;
         const uint32_t buf = (t & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < kStep / 16; ++kk)  // dQ += dS K  (dS of keys 16kk.. at column 16kk)
-            ptx::mma_ts_elect(tmem + 256, tmem + buf + 16 * kk, mnmajor_desc(L::k(sbase, s), kk, kBox64), kIdG,
-                              (t > 0 || kk > 0) ? 1u : 0u);
+        // dQ += dS K  (dS of keys 16kk.. at column 16kk)
+        mma_ts_grad4(tmem + 256, tmem + buf, L::k(sbase, s), kBox64, kIdG, t > 0 ? 1u : 0u);
         ptx::tc_commit_elect(L::bar_empty(sbase, s));
     }
     ptx::tc_commit_elect(L::bar_done(sbase));

@@ -34,31 +34,48 @@ constexpr int kStages = 8;
 // e4m3 products twice as fast, the exponential unit is relieved a little more
 // than in the bf16 kernel (measured: 1/4 beat 1/2, 1/8, 1/16 and none).
 constexpr int kPolyPeriodFp8 = 4;
+// Register split after launch: 128 x (216 + 216 + 72) = 384 x 168 (this
+// kernel's producer and MMA loop need more than the bf16 kernel's 56).
+constexpr uint32_t kRegsSoftmaxFp8 = 216;
+constexpr uint32_t kRegsOtherFp8 = 72;
 
 // kind::f8f6f4 descriptor: e4m3 A and B (format 0), fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
     return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_ss_f8_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
+// The four K-steps of a score product (32 one-byte elements, i.e. +32 bytes
+// = +2 in the descriptor's start field, per step) from one elected lane.
+__device__ __forceinline__ void mma_ss_f8_k4_elect(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
+        "{\n\t.reg .pred f, t, e;\n\t.reg .b64 a, b;\n\t"
         "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "setp.ne.b32 f, %3, %3;\n\t"
+        "setp.eq.b32 t, %3, %3;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, f;\n\t"
+        "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t"
+        "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t"
+        "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t}" ::"r"(d_tmem),
+        "l"(a0), "l"(b0), "r"(idesc)
         : "memory");
 }
 
-__device__ __forceinline__ void mma_ts_f8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
+// Two K-steps of a P V product: A from tensor memory (+8 columns per step), B
+// K-major (+32 bytes per step).
+__device__ __forceinline__ void mma_ts_f8_k2_elect(uint32_t d_tmem, uint32_t a_tmem0, uint64_t b0, uint32_t idesc,
+                                                   uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
         "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t"
+        "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 2;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a], b, %3, t;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem0), "l"(b0), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -206,10 +223,9 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int x, i
     constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, kBN);
     const uint32_t qa = sbase + (x ? L::kQ1 : L::kQ0);
     const uint32_t ka = sbase + L::kKV + slot * kTileBytes;
-#pragma unroll
-    for (int kk = 0; kk < kD / 32; ++kk)  // 32 one-byte elements per step
-        mma_ss_f8_elect(tmem + (x ? 128u : 0u), ptx::smem_desc_sw128(qa + kk * 32, 16, 1024),
-                        ptx::smem_desc_sw128(ka + kk * 32, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
+    static_assert(kD / 32 == 4, "four 32-byte steps cover one 128-byte row");
+    mma_ss_f8_k4_elect(tmem + (x ? 128u : 0u), ptx::smem_desc_sw128(qa, 16, 1024), ptx::smem_desc_sw128(ka, 16, 1024),
+                       kIdesc);
 }
 
 // Keys [128 part / kPParts, 128 (part + 1) / kPParts) of the block.
@@ -219,12 +235,10 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int x, i
     const uint32_t va = sbase + L::kKV + slot * kTileBytes;  // V^T: d rows x 128 keys
     const uint32_t p_tmem = tmem + (x ? 128u : 0u) + kPOffset;
     constexpr int kSteps = kBN / 32 / kPParts;  // 32 keys per step = 8 packed columns of P
-#pragma unroll
-    for (int i = 0; i < kSteps; ++i) {
-        const int kk = part * kSteps + i;
-        mma_ts_f8_elect(tmem + kTmemO0 + (x ? 128u : 0u), p_tmem + kk * 8,
-                        ptx::smem_desc_sw128(va + kk * 32, 16, 1024), kIdesc, (accumulate || i > 0) ? 1u : 0u);
-    }
+    static_assert(kSteps == 2, "two steps per part");
+    const int kk = part * kSteps;
+    mma_ts_f8_k2_elect(tmem + kTmemO0 + (x ? 128u : 0u), p_tmem + kk * 8, ptx::smem_desc_sw128(va + kk * 32, 16, 1024),
+                       kIdesc, accumulate ? 1u : 0u);
 }
 
 // The bf16 kernel's MMA loop (order S0(j), PV1(j-1), S1(j), PV0(j), and its
@@ -453,10 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     if (warp < 8) {
-        ptx::setmaxnreg_inc<kRegsSoftmax>();
+        ptx::setmaxnreg_inc<kRegsSoftmaxFp8>();
         softmax_role(p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
     } else {
-        ptx::setmaxnreg_dec<kRegsOther>();
+        ptx::setmaxnreg_dec<kRegsOtherFp8>();
         if (warp == kWarpProducer)
             producer(p, &tm_q, &tm_k, &tm_vt, sbase, abort_flag);
         else if (warp == kWarpMma)

@@ -503,25 +503,37 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
         kQ = 256u,         // parity of the Q loads consumed
         kUnitShift = 9u,   // bits 9-10: unit queue index mod 4
     };
+    static_assert(kPParts == 2, "the P V product is handed over in two parts");
     uint32_t f = 0;
-    int ring = 0;  // K/V ring slots consumed
-    bool ok = true;
-    // P V of tile x in kPParts parts: part k waits for the softmax's hand-off of
-    // that part (p_part, the last one p_ready); before the first P V of a pair
-    // the first part also waits for the previous pair's epilogue to have read O
-    // (o_free).  Every hand-off barrier completes once per key block.
-    auto pv = [&](int x, int slot, bool last) -> bool {
-#pragma unroll
-        for (int k = 0; k < kPParts; ++k) {
-            const uint32_t bar = k < kPParts - 1 ? L::bar_p_part(sbase, x, k) : L::bar_p_ready(sbase, x);
-            if (!warp_wait(bar, (f >> x) & 1u, abort_flag, lim)) return false;
-            if (k == 0 && (f & (kFirst << x)) && (f & (kPending << x))) {
-                if (!warp_wait(L::bar_o_free(sbase, x), (f >> (4 + x)) & 1u, abort_flag, lim)) return false;
-                f ^= (kFreed << x) | (kPending << x);
-            }
-            ptx::tc_fence_after_sync();
-            issue(x, slot, k, k > 0 || !(f & (kFirst << x)));
+    // Ring position of the next key tile (slot and barrier phase), advanced
+    // one slot at a time: no division on this warp's path.
+    int ks = 0;
+    uint32_t kph = 0;
+    auto adv = [](int& slot, uint32_t& ph) {
+        if (++slot == STAGES) {
+            slot = 0;
+            ph ^= 1u;
         }
+    };
+    bool ok = true;
+    // P V of tile x in two parts: each waits for the softmax's hand-off of its
+    // half of the weights (p_part, then p_ready); before the first P V of a
+    // pair the first part also waits for the previous pair's epilogue to have
+    // read O (o_free).  Every hand-off barrier completes once per key block.
+    // `after_first` runs between the two parts (commits that may block on a
+    // full tensor-core queue go there, behind products already queued).
+    auto pv = [&](int x, int slot, bool last, auto&& after_first) -> bool {
+        if (!warp_wait(L::bar_p_part(sbase, x, 0), (f >> x) & 1u, abort_flag, lim)) return false;
+        if ((f & (kFirst << x)) && (f & (kPending << x))) {
+            if (!warp_wait(L::bar_o_free(sbase, x), (f >> (4 + x)) & 1u, abort_flag, lim)) return false;
+            f ^= (kFreed << x) | (kPending << x);
+        }
+        ptx::tc_fence_after_sync();
+        issue(x, slot, 0, !(f & (kFirst << x)));
+        after_first();
+        if (!warp_wait(L::bar_p_ready(sbase, x), (f >> x) & 1u, abort_flag, lim)) return false;
+        ptx::tc_fence_after_sync();
+        issue(x, slot, 1, true);
         f &= ~(kFirst << x);
         f ^= kPc << x;
         if (last) {
@@ -529,6 +541,21 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
             f |= kPending << x;
         }
         return true;
+    };
+    auto nothing = [] {};
+    // Two ring tiles awaited together: both probes, one vote; the bounded wait
+    // only when one of them is not there yet.
+    auto kv_wait2 = [&](int s0, uint32_t ph0, int s1, uint32_t ph1) -> bool {
+        const bool a = ptx::mbar_try_wait(L::bar_kv_full(sbase, s0), ph0);
+        const bool b = ptx::mbar_try_wait(L::bar_kv_full(sbase, s1), ph1);
+        if (__all_sync(0xffffffffu, a && b)) {
+            ptx::tc_fence_after_sync();
+            return true;
+        }
+        const bool r = warp_wait(L::bar_kv_full(sbase, s0), ph0, abort_flag, lim) &&
+                       warp_wait(L::bar_kv_full(sbase, s1), ph1, abort_flag, lim);
+        ptx::tc_fence_after_sync();
+        return r;
     };
     while (ok) {
         const int u = unit_take<L>(sbase, (f >> kUnitShift) & 3u, abort_flag, lim);
@@ -540,57 +567,68 @@ __device__ __forceinline__ void mma_loop(const FwdParams& p, uint32_t sbase, vol
         f ^= kQ;
         f |= kFirst | (kFirst << 1);
         ptx::tc_fence_after_sync();
+        if (w.uhi <= w.ulo) {
+            ptx::tc_commit_elect(L::bar_q_empty(sbase));  // no products: Q is free
+            continue;
+        }
         // Issue order per key block j:  PV1(j-1), S1(j), PV0(j), S0(j+1), with
         // S0 of the pair's first block before the loop.  Each softmax group
         // then has the two products of the other tile to hide its
         // exponentials behind, and each tile's P V product is followed at once
-        // by its next score product: the value tile of block j and the key
-        // tile of block j+1 are awaited before the tile's weights are, so no
-        // wait sits between the two.  S_x(j) overwrites the P_x(j-1) columns
-        // only after PV_x(j-1) was issued; tcgen05 MMAs from one thread
-        // execute in order.
-        if (w.uhi > w.ulo) {
-            const int ks = ring % STAGES;
-            if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), (ring / STAGES) & 1, abort_flag, lim))) break;
-            ptx::tc_fence_after_sync();
-            if (w.ulo >= lo0 && w.ulo < hi0) {
-                qk(0, ks);
-                ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
-            }
+        // by its next score product.  This warp's waits and commits sit where
+        // a score product (512 tensor cycles) has just been queued: the value
+        // tile of block j and the key tile of block j+1 are awaited together
+        // after S1(j), and the key tile's release goes out behind PV0(j).  S_x(j) overwrites the P_x(j-1) columns only after
+        // PV_x(j-1) was issued; tcgen05 MMAs from one thread execute in order.
+        if (!(ok = warp_wait(L::bar_kv_full(sbase, ks), kph, abort_flag, lim))) break;
+        ptx::tc_fence_after_sync();
+        if (w.ulo >= lo0 && w.ulo < hi0) {
+            qk(0, ks);
+            ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
         }
-        for (int j = w.ulo; ok && j < w.uhi; ++j, ring += 2) {
-            const int ks = ring % STAGES, vs = (ring + 1) % STAGES, nks = (ring + 2) % STAGES;
+        int pvs = 0;  // ring slot of the previous block's value tile
+        for (int j = w.ulo; j < w.uhi; ++j) {
+            int vs = ks;
+            uint32_t vph = kph;
+            adv(vs, vph);
+            int nks = vs;
+            uint32_t nph = vph;
+            adv(nks, nph);
+            const bool more = j + 1 < w.uhi;
             if (j > w.ulo) {
-                const int pvs = (ring - 1) % STAGES;
-                if (j - 1 >= lo1 && j - 1 < hi1 && !(ok = pv(1, pvs, j - 1 == hi1 - 1))) break;
+                if (j - 1 >= lo1 && j - 1 < hi1 && !(ok = pv(1, pvs, j - 1 == hi1 - 1, nothing))) break;
                 ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
             }
             if (j >= lo1 && j < hi1) {
                 qk(1, ks);
                 ptx::tc_commit_elect(L::bar_s_full(sbase, 1));
             }
-            ptx::tc_commit_elect(L::bar_kv_empty(sbase, ks));
-            if (j == w.uhi - 1) ptx::tc_commit_elect(L::bar_q_empty(sbase));  // last score products issued
-            const bool more = j + 1 < w.uhi;
-            if (!(ok = warp_wait(L::bar_kv_full(sbase, vs), ((ring + 1) / STAGES) & 1, abort_flag, lim))) break;
-            if (more && !(ok = warp_wait(L::bar_kv_full(sbase, nks), ((ring + 2) / STAGES) & 1, abort_flag, lim)))
-                break;
-            ptx::tc_fence_after_sync();
-            if (j >= lo0 && j < hi0 && !(ok = pv(0, vs, j == hi0 - 1))) break;
+            // value tile j and key tile j+1 (loaded well ahead): one wait for both,
+            // while the score product just issued keeps the tensor pipe busy
+            if (!(ok = kv_wait2(vs, vph, more ? nks : vs, more ? nph : vph))) break;
+            // the key tile of block j is free once both score products are out
+            const int kslot = ks;
+            auto release_k = [&] {
+                ptx::tc_commit_elect(L::bar_kv_empty(sbase, kslot));
+                if (j == w.uhi - 1) ptx::tc_commit_elect(L::bar_q_empty(sbase));  // last score products issued
+            };
+            if (j >= lo0 && j < hi0) {
+                if (!(ok = pv(0, vs, j == hi0 - 1, release_k))) break;
+            } else {
+                release_k();
+            }
             if (more && j + 1 >= lo0 && j + 1 < hi0) {
                 qk(0, nks);
                 ptx::tc_commit_elect(L::bar_s_full(sbase, 0));
             }
+            pvs = vs;
+            ks = nks;
+            kph = nph;
         }
         if (!ok) break;
-        if (w.uhi > w.ulo) {
-            const int j = w.uhi - 1;
-            const int vs = (ring - 1) % STAGES;
-            if (j >= lo1 && j < hi1 && !(ok = pv(1, vs, true))) break;
-            ptx::tc_commit_elect(L::bar_kv_empty(sbase, vs));
-        } else {
-            ptx::tc_commit_elect(L::bar_q_empty(sbase));  // no products: Q is free
-        }
+        const int j = w.uhi - 1;
+        if (j >= lo1 && j < hi1 && !(ok = pv(1, pvs, true, nothing))) break;
+        ptx::tc_commit_elect(L::bar_kv_empty(sbase, pvs));
     }
     // All MMAs must be complete before tensor memory is released.
     ptx::tc_commit_elect(L::bar_mma_final(sbase));
