@@ -123,6 +123,7 @@ struct Layout {
     static constexpr uint32_t kUnitQ = kClcResp + 16;       // unit queue: two ints
     static constexpr uint32_t kBytes = kUnitQ + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
+    static_assert(kClcResp % 16 == 0, "the launch-control response needs 16-byte alignment");
 
     static __device__ __forceinline__ uint32_t bar_q(uint32_t base) { return base + kBar; }
     static __device__ __forceinline__ uint32_t bar_kv_full(uint32_t base, int s) { return base + kBar + 8u * (1 + s); }
