@@ -1154,7 +1154,7 @@ def main_ring(args, rank, world, local_rank):
                          "frac": achieved / peak, "traffic": None,
                          "peak_source": f"{src} bf16_tflops (burst, cuBLAS)" if src == "measured"
                          else "fallback 1590 TF/s",
-                         "kernel": "attn_fwd_sm100<128,5,accumulate> + attn_acc_to_bf16",
+                         "kernel": "attn_fwd_sm100<128,4,accumulate> + attn_acc_to_bf16",
                          "timed_as": "whole ring step per rank (all chunk pairs, transfers, cast)"},
             "clocks": clocks,
         }), flush=True)
@@ -1502,7 +1502,7 @@ def main():
                          else "fallback 1590 TF/s",
                          "frac_of_sustained": (achieved / sustained) if sustained else None,
                          "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
-                         "kernel": "attn_fwd_sm100<128,5>" if w.d == 128 else "attn_fwd_sm100<64,8>"},
+                         "kernel": "attn_fwd_sm100<128,4>" if w.d == 128 else "attn_fwd_sm100<64,8>"},
             "clocks": clocks,
             "step_ms": step_stats(run_cuda.step_times),
         }

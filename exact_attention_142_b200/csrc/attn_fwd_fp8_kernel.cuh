@@ -114,7 +114,9 @@ struct Layout {
     static constexpr uint32_t kQ0 = 0;
     static constexpr uint32_t kQ1 = kTileBytes;
     static constexpr uint32_t kKV = 2 * kTileBytes;
-    static constexpr uint32_t kBar = kKV + kStages * kTileBytes;
+    // Output staging: 4 KB per softmax warp (32 rows x 64 bf16 columns).
+    static constexpr uint32_t kStg = kKV + kStages * kTileBytes;
+    static constexpr uint32_t kBar = kStg + 8 * 4096;
     // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
     // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_part[2][kPParts - 1]
     static constexpr uint32_t kNumBars = 16 + 2 * (kPParts - 1) + 2 * kStages;
@@ -386,21 +388,8 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
     const int h = x ? we.h[1] : we.h[0];
     const bool store = row < we.len;
     const float inv = l_q > 0.0f ? 1.0f / l_q : 0.0f;
-    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)(we.start + (store ? row : 0)) * p.Hq + h) * (size_t)kD * 2;
-#pragma unroll
-    for (int cc = 0; cc < kD / 32; ++cc) {
-        uint32_t o[32];
-        ptx::tmem_ld32_sync(t_o + cc * 32, o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            pk[i] = ptx::pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (store) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-                ptx::st_global_v4(orow + cc * 64 + v * 16, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-    }
+    store_o_rows<kD>(p, sbase + L::kStg + (uint32_t)(x * 4 + warp_in_group) * 4096u, lane, t_o, inv,
+                     r0 + warp_in_group * 32, we.len, we.start, h);
     if (store) {
         const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
         const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + row : ((size_t)we.b * p.Hq + h) * p.N + row;

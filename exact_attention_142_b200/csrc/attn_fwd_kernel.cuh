@@ -127,7 +127,9 @@ struct SmemLayout {
     static constexpr uint32_t kQ0 = 0;
     static constexpr uint32_t kQ1 = kTileBytes;
     static constexpr uint32_t kKV = 2 * kTileBytes;
-    static constexpr uint32_t kBar = kKV + STAGES * kTileBytes;
+    // Output staging: 4 KB per softmax warp (32 rows x 64 bf16 columns).
+    static constexpr uint32_t kStg = kKV + STAGES * kTileBytes;
+    static constexpr uint32_t kBar = kStg + 8 * 4096;
     // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_final,
     // q_empty, o_free[2], clc, unit_full[2], unit_empty[2], p_part[2][kPParts - 1]
     static constexpr uint32_t kNumBars = 16 + 2 * (kPParts - 1) + 2 * STAGES;
@@ -443,6 +445,50 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensor
     if (units > 0) drain_wait(L::bar_q(sbase), (units - 1) & 1, lim);
     const int first = issued > STAGES ? issued - STAGES : 0;
     for (int i = first; i < issued; ++i) drain_wait(L::bar_kv_full(sbase, i % STAGES), (i / STAGES) & 1, lim);
+}
+
+// ---------------------------------------------------------------- O stores
+// Writes one softmax warp's 32 rows of O (d fp32 columns of tensor memory at
+// t_o, this thread's row in its lane, times inv, rounded to bf16) to
+// o[start + row][h][:].  They pass through the warp's 4 KB staging area
+// (stg), 64 columns at a time: each thread writes its row's 128 bytes there
+// (16-byte chunks rotated by the row: conflict-free), then each of the warp's
+// eight store instructions writes four whole 128-byte row segments.  Rows at
+// or past len (a packed sequence's end) are not written.
+template <int D>
+__device__ __forceinline__ void store_o_rows(const FwdParams& p, uint32_t stg, int lane, uint32_t t_o, float inv,
+                                             int rbase, int len, int start, int h) {
+#pragma unroll
+    for (int hf = 0; hf < D / 64; ++hf) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            uint32_t o[32];
+            ptx::tmem_ld32_sync(t_o + hf * 64 + cc * 32, o);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int ch = cc * 4 + c;
+                ptx::st_shared_v4(stg + lane * 128 + ((ch ^ (lane & 7)) << 4),
+                                  ptx::pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
+                                  ptx::pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
+                                  ptx::pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
+                                  ptx::pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            const int ch = lane & 7;
+            uint32_t a, b, c, d;
+            ptx::ld_shared_v4(stg + r * 128 + ((ch ^ (r & 7)) << 4), a, b, c, d);
+            if (rbase + r < len) {
+                uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) +
+                               ((size_t)(start + rbase + r) * p.Hq + h) * (size_t)D * 2 + hf * 128 + ch * 16;
+                ptx::st_global_v4(dst, a, b, c, d);
+            }
+        }
+        __syncwarp();  // the staging area is rewritten for the next 64 columns
+    }
 }
 
 // ---------------------------------------------------------------- MMA issuer
@@ -842,23 +888,8 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
         return true;
     }
     const float inv = l_bf > 0.0f ? 1.0f / l_bf : 0.0f;
-    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
-                    ((size_t)(we.start + (store ? row : 0)) * p.Hq + h) * (size_t)D * 2;
-#pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        ptx::tmem_ld32_sync(t_o + cc * 32, o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            pk[i] = ptx::pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (store) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-                ptx::st_global_v4(orow + cc * 64 + v * 16, pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
-                                  pk[4 * v + 3]);
-        }
-    }
+    store_o_rows<D>(p, sbase + L::kStg + (uint32_t)(x * 4 + warp_in_group) * 4096u, lane, t_o, inv,
+                    r0 + warp_in_group * 32, we.len, we.start, h);
     if (store) {
         const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
         const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + row
