@@ -41,14 +41,15 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, cols] bf16, row stride cols * 2 bytes; boxes of 128 rows x 64 columns
-// (128 bytes) with 128-byte swizzling.  Rows past the end read as zero.
-bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+// [rows, cols] bf16, row stride cols * 2 bytes; boxes of box_rows rows x 64
+// columns (128 bytes) with 128-byte swizzling: 128 rows for the Q, K, V loads
+// (rows past the end read as zero), 32 for the output stores of one warp.
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows = 128) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estride[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -148,10 +149,10 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
 // not started (the kernel's persistent schedule), so only about one CTA per
 // SM ever runs.
 template <int D, int STAGES, bool ACC>
-int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-           long long units, cudaStream_t stream) {
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+           const FwdParams& p, long long units, cudaStream_t stream) {
     attn::attn_fwd_sm100<D, STAGES, ACC><<<(unsigned)units, attn::kThreads,
-                                            attn::SmemLayout<D, STAGES>::kDynamicBytes, stream>>>(mq, mk, mv, p);
+                                            attn::SmemLayout<D, STAGES>::kDynamicBytes, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -174,10 +175,12 @@ int run_fwd(bool acc, const void* q, const void* k, const void* v, void* o, floa
     rc = prepare_device(d);
     if (rc != ATTN_OK) return rc;
 
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, (uint64_t)tokens, (uint64_t)Hq * d) ||
         !make_map(&mk, k, (uint64_t)tokens, (uint64_t)Hkv * d) ||
-        !make_map(&mv, v, (uint64_t)tokens, (uint64_t)Hkv * d))
+        !make_map(&mv, v, (uint64_t)tokens, (uint64_t)Hkv * d) ||
+        // O, stored per warp; the accumulating epilogue (fp32 o) does not use it
+        !make_map(&mo, acc ? q : o, (uint64_t)tokens, (uint64_t)Hq * d, 32))
         return ATTN_ERR_CUDA;
 
     FwdParams p;
@@ -204,10 +207,10 @@ int run_fwd(bool acc, const void* q, const void* k, const void* v, void* o, floa
     if (units <= 0) return ATTN_OK;
     if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
     if (acc)
-        return d == 128 ? launch<128, kStages128, true>(mq, mk, mv, p, units, s)
-                        : launch<64, kStages64, true>(mq, mk, mv, p, units, s);
-    return d == 128 ? launch<128, kStages128, false>(mq, mk, mv, p, units, s)
-                    : launch<64, kStages64, false>(mq, mk, mv, p, units, s);
+        return d == 128 ? launch<128, kStages128, true>(mq, mk, mv, mo, p, units, s)
+                        : launch<64, kStages64, true>(mq, mk, mv, mo, p, units, s);
+    return d == 128 ? launch<128, kStages128, false>(mq, mk, mv, mo, p, units, s)
+                    : launch<64, kStages64, false>(mq, mk, mv, mo, p, units, s);
 }
 
 }  // namespace

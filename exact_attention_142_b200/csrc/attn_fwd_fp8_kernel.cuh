@@ -388,8 +388,10 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
     const int h = x ? we.h[1] : we.h[0];
     const bool store = row < we.len;
     const float inv = l_q > 0.0f ? 1.0f / l_q : 0.0f;
+    // Row-segment stores from the staging area: TMA box stores measured 4 %
+    // slower in this kernel (0.822 -> 0.855 ms on the 8192-token GQA workload).
     store_o_rows<kD>(p, sbase + L::kStg + (uint32_t)(x * 4 + warp_in_group) * 4096u, lane, t_o, inv,
-                     r0 + warp_in_group * 32, we.len, we.start, h);
+                     r0 + warp_in_group * 32, we.len, we.start, h, nullptr);
     if (store) {
         const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
         const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + row : ((size_t)we.b * p.Hq + h) * p.N + row;

@@ -450,14 +450,20 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const CUtensor
 // ---------------------------------------------------------------- O stores
 // Writes one softmax warp's 32 rows of O (d fp32 columns of tensor memory at
 // t_o, this thread's row in its lane, times inv, rounded to bf16) to
-// o[start + row][h][:].  They pass through the warp's 4 KB staging area
-// (stg), 64 columns at a time: each thread writes its row's 128 bytes there
-// (16-byte chunks rotated by the row: conflict-free), then each of the warp's
-// eight store instructions writes four whole 128-byte row segments.  Rows at
-// or past len (a packed sequence's end) are not written.
+// o[start + row][h][:].  They pass through the warp's 4 KB staging area (stg,
+// 1 KB aligned), 64 columns at a time: each thread writes its row's 128 bytes
+// there with the 16-byte chunks rotated by the row (chunk c of row r at
+// c ^ (r mod 8): conflict-free, and the 128-byte swizzle of a TMA box).  When
+// all 32 rows lie inside the sequence, one lane stores the staging area as a
+// 32 x 64 box through tm_o (the copy engine writes O; no load/store-unit
+// traffic) and waits until the copy has read it before the next 64 columns
+// are staged.  Otherwise (a warp that reaches past a packed sequence's end, or
+// no map) each of the warp's eight store instructions writes four whole
+// 128-byte row segments, and rows at or past len are skipped.
 template <int D>
 __device__ __forceinline__ void store_o_rows(const FwdParams& p, uint32_t stg, int lane, uint32_t t_o, float inv,
-                                             int rbase, int len, int start, int h) {
+                                             int rbase, int len, int start, int h, const CUtensorMap* tm_o) {
+    const bool box = tm_o != nullptr && rbase + 32 <= len;
 #pragma unroll
     for (int hf = 0; hf < D / 64; ++hf) {
 #pragma unroll
@@ -473,6 +479,17 @@ __device__ __forceinline__ void store_o_rows(const FwdParams& p, uint32_t stg, i
                                   ptx::pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
                                   ptx::pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
             }
+        }
+        if (box) {
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::tma_store_2d(tm_o, stg, h * D + hf * 64, start + rbase);
+                ptx::bulk_commit_group();
+                ptx::bulk_wait_group_read0();
+            }
+            __syncwarp();
+            continue;
         }
         __syncwarp();
 #pragma unroll
@@ -698,7 +715,8 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
 template <int D, int STAGES, bool ACC>
 __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams& p, int x,
                                              int warp_in_group, int lane, uint32_t tmem,
-                                             uint32_t sbase, volatile int* abort_flag, uint32_t& phases, int u) {
+                                             uint32_t sbase, volatile int* abort_flag, uint32_t& phases, int u,
+                                             const CUtensorMap* tm_o) {
     using L = SmemLayout<D, STAGES>;
     const int r0 = x ? w.r0[1] : w.r0[0];
     const int blk_lo = x ? w.lo[1] : w.lo[0];
@@ -889,7 +907,7 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
     }
     const float inv = l_bf > 0.0f ? 1.0f / l_bf : 0.0f;
     store_o_rows<D>(p, sbase + L::kStg + (uint32_t)(x * 4 + warp_in_group) * 4096u, lane, t_o, inv,
-                    r0 + warp_in_group * 32, we.len, we.start, h);
+                    r0 + warp_in_group * 32, we.len, we.start, h, tm_o);
     if (store) {
         const float lse = l_sum > 0.0f ? (m_ref + ptx::lg2_approx(l_sum)) * kLn2 : -INFINITY;
         const size_t idx = p.cu_seqlens ? (size_t)h * p.N + we.start + row
@@ -905,7 +923,8 @@ __device__ __forceinline__ bool softmax_unit(const TilePair& w, const FwdParams&
 // The units of this CTA for one tile of the pair (tiles with no rows skipped).
 template <int D, int STAGES, bool ACC>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, int x, int warp_in_group, int lane,
-                                             uint32_t tmem, uint32_t sbase, volatile int* abort_flag) {
+                                             uint32_t tmem, uint32_t sbase, volatile int* abort_flag,
+                                             const CUtensorMap* tm_o) {
     // bit 0: s_full parity, bit 1: o_done parity, bits 2-3: unit queue index mod 4
     uint32_t phases = 0;
     while (true) {
@@ -914,17 +933,19 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, int x, int warp
         if (u < 0) break;
         const TilePair w = decode_pair(u, p);
         if (!(x ? w.active[1] : w.active[0])) continue;
-        if (!softmax_unit<D, STAGES, ACC>(w, p, x, warp_in_group, lane, tmem, sbase, abort_flag, phases, u))
-            return;
+        if (!softmax_unit<D, STAGES, ACC>(w, p, x, warp_in_group, lane, tmem, sbase, abort_flag, phases, u, tm_o))
+            break;
         phases ^= 2u;
     }
+    if (lane == 0) ptx::bulk_wait_group0();  // this warp's output copies are complete
 }
 
 // ---------------------------------------------------------------- kernel
 template <int D, int STAGES, bool ACC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const FwdParams p) {
     using L = SmemLayout<D, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -954,6 +975,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tensormap(&tm_q);
         ptx::prefetch_tensormap(&tm_k);
         ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_o);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
@@ -966,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
-        softmax_role<D, STAGES, ACC>(p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag);
+        softmax_role<D, STAGES, ACC>(p, warp / 4, warp % 4, lane, tmem, sbase, abort_flag, ACC ? nullptr : &tm_o);
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (warp == kWarpProducer) {
