@@ -679,13 +679,6 @@ struct DqLayout {
     static __device__ __forceinline__ uint32_t bar_a(uint32_t base) { return base + kBar + 8u * (6 + 2 * STAGES); }
 };
 
-__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
-                 : "r"(addr)
-                 : "memory");
-}
-
 // Copies this thread's row of Q (groups 0, 1) or dO (groups 2, 3) from the
 // TMA tile (128-byte swizzle: 16-byte chunk c of row r sits at chunk
 // c ^ (r mod 8) of its 128-byte line) into tensor memory, half a row per
@@ -701,7 +694,7 @@ __device__ __forceinline__ void dq_stage_a(uint32_t tl, uint32_t sbase, int x, i
     for (int i = 0; i < kChunks; ++i) {
         const int c = c0 + i;
         const uint32_t addr = src + (c >> 3) * kBox128 + row * 128 + (((c & 7) ^ (row & 7)) << 4);
-        ld_shared_v4(addr, r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+        ptx::ld_shared_v4(addr, r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
     }
     const uint32_t dst = tl + (x < 2 ? L::kTQ : L::kTDO) + 4 * c0;
     if constexpr (kChunks == 8)
